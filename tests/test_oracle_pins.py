@@ -1,0 +1,404 @@
+"""Pins for the CPU oracle: facts fixed by the pages and by mathematics, not by
+the oracle's own code.
+
+Sources: ECF8 walkthrough ("ECF8 浮点数压缩技术") p1 §1 (bit-exact), §3.1.1
+(per-layer exponent statistics, optimal prefix code, length <= 16), §3.1.2
+(decode table), §3.2.1 (per-thread gap), §5.3 (gap synchronisation as the
+failure mode); arXiv 2510.02676 abstract (lossless, "no deviation").
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import ecf8_synth as synth
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def _kraft(lengths):
+    return sum(2.0 ** -int(l) for l in lengths if l)
+
+
+def _entropy_bits(hist):
+    h = np.asarray(hist, dtype=np.float64)
+    p = h[h > 0] / h.sum()
+    return float(-(p * np.log2(p)).sum())
+
+
+# ---------------------------------------------------------------- split / join
+
+def test_split_matches_e4m3_value_meaning():
+    """The exponent field and nibble reproduce the E4M3 value that torch decodes:
+    (-1)^s 2^(e-7) (1 + m/8) for e >= 1 and (-1)^s 2^-6 (m/8) for e = 0."""
+    vals = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    for b in range(256):
+        e, nib = oracle.exponent(b), oracle.nibble(b)
+        s, m = nib >> 3, nib & 7
+        if b in (0x7F, 0xFF):
+            assert math.isnan(vals[b])
+            continue
+        mag = 2.0 ** (e - 7) * (1 + m / 8) if e else 2.0 ** -6 * (m / 8)
+        assert vals[b] == (-mag if s else mag), b
+        assert oracle.join(e, nib) == b
+
+
+# ---------------------------------------------------------------- code construction
+
+def _random_hists(count, k_max=16, seed=1):
+    r = _rng(seed)
+    for _ in range(count):
+        k = int(r.integers(1, k_max + 1))
+        syms = r.choice(16, size=k, replace=False)
+        h = np.zeros(16, dtype=np.uint64)
+        scale = 10 ** int(r.integers(0, 7))
+        h[syms] = r.integers(1, scale + 1, size=k)
+        yield h
+
+
+def _is_prefix_free(lengths, codes):
+    words = [format(int(codes[s]), f"0{int(lengths[s])}b") for s in range(16) if lengths[s]]
+    for a, b in itertools.permutations(words, 2):
+        if b.startswith(a):
+            return False
+    return len(set(words)) == len(words)
+
+
+def test_prefix_free_kraft_and_length_limit():
+    for h in _random_hists(400):
+        ln = oracle.code_lengths(h)
+        k = int((h > 0).sum())
+        assert all((ln[s] > 0) == (h[s] > 0) for s in range(16))
+        assert ln.max() <= 15  # 16 leaves cannot be deeper; within the page's 16-bit cap
+        codes = oracle.canonical_codes(ln)
+        assert _is_prefix_free(ln, codes)
+        if k >= 2:
+            assert _kraft(ln) == 1.0  # a Huffman code is complete
+        else:
+            assert list(ln[h > 0]) == [1]
+
+
+def _brute_min_cost(weights, max_len):
+    """Minimum sum w*l over all length vectors with Kraft <= 1 and l <= max_len."""
+    k = len(weights)
+    best = None
+    for ls in itertools.product(range(1, max_len + 1), repeat=k):
+        if sum(2.0 ** -l for l in ls) <= 1.0:
+            c = sum(w * l for w, l in zip(weights, ls))
+            best = c if best is None or c < best else best
+    return best
+
+
+@pytest.mark.parametrize("k", [2, 3, 4, 5, 6])
+def test_huffman_optimal_by_brute_force(k):
+    r = _rng(k)
+    for _ in range(25 if k < 6 else 8):
+        h = np.zeros(16, dtype=np.uint64)
+        syms = r.choice(16, size=k, replace=False)
+        h[syms] = r.integers(1, 50, size=k)
+        ln = oracle.huffman_lengths(h)
+        cost = int(sum(int(h[s]) * int(ln[s]) for s in range(16)))
+        assert cost == _brute_min_cost([int(h[s]) for s in syms], k - 1)
+
+
+@pytest.mark.parametrize("k,limit", [(4, 2), (5, 3), (6, 3), (6, 4), (7, 3)])
+def test_package_merge_optimal_under_limit(k, limit):
+    r = _rng(100 + k * 10 + limit)
+    for _ in range(20 if k < 7 else 6):
+        h = np.zeros(16, dtype=np.uint64)
+        syms = r.choice(16, size=k, replace=False)
+        h[syms] = r.integers(1, 1000, size=k) ** 2  # skewed, so the limit binds
+        ln = oracle.package_merge_lengths(h, limit)
+        assert ln.max() <= limit and _kraft(ln) <= 1.0
+        cost = int(sum(int(h[s]) * int(ln[s]) for s in range(16)))
+        assert cost == _brute_min_cost([int(h[s]) for s in syms], limit)
+
+
+def test_package_merge_equals_huffman_cost_when_limit_is_loose():
+    for h in _random_hists(100, seed=7):
+        a, b = oracle.huffman_lengths(h), oracle.package_merge_lengths(h, 16)
+        assert int((h * a.astype(np.uint64)).sum()) == int((h * b.astype(np.uint64)).sum())
+
+
+def test_length_limit_is_infeasible_below_log2_k():
+    h = np.ones(16, dtype=np.uint64)
+    with pytest.raises(ValueError):
+        oracle.code_lengths(h, max_len=3)
+    assert list(oracle.code_lengths(h, max_len=4)) == [4] * 16
+
+
+def test_entropy_bounds_shannon():
+    """n H <= sum f l < n (H + 1) for the optimal code."""
+    for h in _random_hists(300, seed=3):
+        n = int(h.sum())
+        k = int((h > 0).sum())
+        ln = oracle.code_lengths(h)
+        bits = int((h * ln.astype(np.uint64)).sum())
+        H = _entropy_bits(h)
+        if k >= 2:
+            assert n * H <= bits + 1e-6 * n
+        assert bits < n * (H + 1) + 1e-9 * n
+
+
+def test_fibonacci_frequencies_give_the_deepest_code():
+    """Fibonacci weights force a chain: lengths 15,15,14,...,1 and codes
+    (L-1 ones then a zero) -- the longest code 16 symbols allow."""
+    fib = [1, 1]
+    while len(fib) < 16:
+        fib.append(fib[-1] + fib[-2])
+    h = np.array(fib, dtype=np.uint64)
+    ln = oracle.code_lengths(h)
+    assert list(ln) == [15, 15] + [16 - s for s in range(2, 16)]
+    codes = oracle.canonical_codes(ln)
+    assert int(codes[15]) == 0
+    for s in range(2, 15):
+        L = 16 - s
+        assert int(codes[s]) == (1 << L) - 2
+    assert int(codes[0]) == 0x7FFE and int(codes[1]) == 0x7FFF
+
+
+def test_single_symbol_gets_one_bit():
+    h = np.zeros(16, dtype=np.uint64)
+    h[5] = 1000
+    ln = oracle.code_lengths(h)
+    assert ln[5] == 1 and ln.sum() == 1
+    assert int(oracle.canonical_codes(ln)[5]) == 0
+
+
+# ---------------------------------------------------------------- closed-form streams
+
+def _stream_words(blob):
+    hd = oracle.blob_header(blob)
+    words = (hd["code_bits"] + 31) // 32
+    return blob[hd["stream_off"]: hd["stream_off"] + 4 * words].view("<u4"), hd
+
+
+def test_uniform_16_symbols_stream_is_the_packed_exponents():
+    """All 16 exponents equally frequent: every code is 4 bits and code(e) = e,
+    so the stream is the exponent fields themselves, MSB first."""
+    r = _rng(11)
+    e = np.tile(np.arange(16, dtype=np.uint8), 64)
+    r.shuffle(e)
+    nib = r.integers(0, 16, size=e.size).astype(np.uint8)
+    x = ((nib >> 3) << 7) | (e << 3) | (nib & 7)
+    blob = oracle.encode(x)
+    words, hd = _stream_words(blob)
+    assert list(hd["lengths"]) == [4] * 16
+    want = np.zeros(e.size // 8, dtype=np.uint32)
+    for i, v in enumerate(e):
+        want[i // 8] |= np.uint32(int(v) << (28 - 4 * (i % 8)))
+    assert np.array_equal(words, want)
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+
+
+def test_two_symbols_stream_is_a_bitmap():
+    r = _rng(12)
+    e = np.where(r.random(1000) < 0.3, 9, 4).astype(np.uint8)
+    x = (e << 3) | 5
+    blob = oracle.encode(x)
+    words, hd = _stream_words(blob)
+    assert hd["lengths"][4] == 1 and hd["lengths"][9] == 1
+    bits = "".join("1" if v == 9 else "0" for v in e)
+    bits += "0" * (-len(bits) % 32)
+    want = np.array([int(bits[i:i + 32], 2) for i in range(0, len(bits), 32)], dtype=np.uint32)
+    assert np.array_equal(words, want)
+
+
+# ---------------------------------------------------------------- worked example (hand-derived)
+
+def _read_golden(name):
+    d = {"lut": []}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            if key == "lut":
+                d["lut"].append((int(vals[0], 16), int(vals[1], 16)))
+            else:
+                d[key] = vals
+    return d
+
+
+def test_hand_worked_example():
+    g = _read_golden("worked_example.txt")
+    x = np.array([int(v, 16) for v in g["weights"]], dtype=np.uint8)
+    C, T = int(g["chunk_bytes"][0]), int(g["group_chunks"][0])
+    hist = oracle.histogram(x)
+    ln = oracle.code_lengths(hist)
+    assert list(ln) == [int(v) for v in g["lengths"]]
+    codes = oracle.canonical_codes(ln)
+    assert [int(c) if l else 0 for c, l in zip(codes, ln)] == [int(v) for v in g["codes"]]
+    blob = oracle.encode(x, chunk_bytes=C, group_chunks=T)
+    hd = oracle.blob_header(blob)
+    assert hd["code_bits"] == int(g["code_bits"][0])
+    assert hd["n_groups"] == int(g["n_groups"][0])
+    sw = blob[hd["stream_off"]:hd["stream_off"] + 8].view("<u4")
+    assert [int(w) for w in sw] == [int(v, 16) for v in g["stream_words"]]
+    gw = blob[hd["gaps_off"]:hd["gaps_off"] + 4].view("<u4")
+    assert [int(w) for w in gw] == [int(v, 16) for v in g["gap_words"]]
+    go = blob[hd["groups_off"]:hd["groups_off"] + 8 * 3].view("<u8")
+    assert [int(w) for w in go] == [int(v) for v in g["group_offsets"]]
+    nb = blob[hd["nibbles_off"]:hd["nibbles_off"] + 16]
+    assert [int(v) for v in nb] == [int(v, 16) for v in g["nibble_bytes"]]
+    lut = blob[hd["lut_off"]:hd["lut_off"] + 4 * 4096].view("<u4")
+    for pat, want in g["lut"]:
+        assert int(lut[pat]) == want, hex(pat)
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+
+
+# ---------------------------------------------------------------- decode table
+
+def test_decode_table_entries_are_greedy_and_maximal():
+    """Each entry's codes spell exactly its first `used` bits, and either it holds
+    6 codes or no code fits in the bits left over -- this fixes every entry."""
+    for h in list(_random_hists(6, seed=21)) + [np.array([1, 1] + [0] * 14, dtype=np.uint64)]:
+        ln = oracle.code_lengths(h)
+        codes = oracle.canonical_codes(ln)
+        words = {s: format(int(codes[s]), f"0{int(ln[s])}b") for s in range(16) if ln[s]}
+        for pat in range(4096):
+            e = oracle.lut_entry(ln, pat)
+            used, cnt = e & 15, (e >> 4) & 7
+            syms = [(e >> (8 + 4 * j)) & 15 for j in range(cnt)]
+            assert e >> (8 + 4 * cnt) == 0 and (e >> 7) & 1 == 0
+            bits = format(pat, "012b")
+            spelled = "".join(words[s] for s in syms)
+            assert spelled == bits[:used] and len(spelled) == used
+            rest = bits[used:]
+            if cnt < 6:
+                assert not any(rest.startswith(w) for w in words.values())
+
+
+# ---------------------------------------------------------------- round trip (the definition)
+
+EDGE_SIZES = [0, 1, 2, 3, 7, 8, 31, 32, 33, 4095, 4096, 4097]
+
+
+@pytest.mark.parametrize("n", EDGE_SIZES)
+def test_round_trip_edge_sizes(n):
+    x = synth.single_normal_1k().tensors[0].generate(count=n) if n else np.zeros(0, np.uint8)
+    for C, T in [(32, 128), (4, 1), (16, 3)]:
+        blob = oracle.encode(x, chunk_bytes=C, group_chunks=T)
+        assert np.array_equal(oracle.decode(blob, n), x)
+        assert oracle.check_index(blob) == 0
+
+
+def test_round_trip_every_byte_value_and_specials():
+    r = _rng(5)
+    base = np.arange(256, dtype=np.uint8)
+    x = np.concatenate([base, r.permutation(np.repeat(base, 40)), np.array([0x7F, 0xFF, 0x00, 0x80] * 9, np.uint8)])
+    blob = oracle.encode(x)
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+    assert oracle.check_index(blob) == 0
+
+
+def test_round_trip_uniform_random_bytes_is_lossless_even_when_it_expands():
+    x = _rng(6).integers(0, 256, size=100_000).astype(np.uint8)
+    blob = oracle.encode(x)
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+    assert blob.size > x.size  # 4 code bits + 4 nibble bits + index: no raw fallback
+
+
+def test_round_trip_single_symbol_and_deepest_code():
+    x = np.full(5000, 0x38, dtype=np.uint8)
+    blob = oracle.encode(x)
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+    fib = [1, 1]
+    while len(fib) < 16:
+        fib.append(fib[-1] + fib[-2])
+    e = np.repeat(np.arange(16, dtype=np.uint8), fib)
+    e = _rng(9).permutation(e)
+    x = (e << 3) | (_rng(10).integers(0, 8, size=e.size).astype(np.uint8))
+    blob = oracle.encode(x)
+    assert oracle.blob_header(blob)["max_len"] == 15
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+    assert oracle.check_index(blob) == 0
+
+
+@pytest.mark.parametrize("max_len", [4, 5, 6, 8])
+def test_round_trip_with_binding_length_limit(max_len):
+    x = synth.alpha_sweep_point(1.5, 448.0).tensors[0].generate(count=200_000)
+    blob = oracle.encode(x, max_len=max_len)
+    assert oracle.blob_header(blob)["max_len"] <= max_len
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+
+
+# ---------------------------------------------------------------- gap synchronisation (p1 §5.3)
+
+def test_corrupt_gap_and_offset_are_detected():
+    x = synth.single_normal_1k().tensors[0].generate(count=300_000)
+    blob = oracle.encode(x)
+    hd = oracle.blob_header(blob)
+    bad = blob.copy()
+    bad[hd["gaps_off"] + 5] ^= 0x10
+    assert oracle.check_index(bad) == 2
+    bad = blob.copy()
+    bad[hd["groups_off"] + 8] ^= 1
+    assert oracle.check_index(bad) == 3
+    bad = blob.copy()
+    bad[hd["lut_off"] + 4 * 77] ^= 0x20
+    assert oracle.check_index(bad) == 1
+    bad = blob.copy()
+    bad[0] ^= 1
+    with pytest.raises(ValueError):
+        oracle.decode(bad, x.size)
+
+
+# ---------------------------------------------------------------- synthetic inputs
+
+def test_generator_cast_matches_torch_e4m3():
+    r = _rng(13)
+    v = np.concatenate([r.standard_normal(50_000) * 40, r.standard_normal(50_000) * 0.01,
+                        np.array([0.0, -0.0, 448.0, -448.0, 2 ** -9, 2 ** -10, 1.5 * 2 ** -10])])
+    v = np.clip(v.astype(np.float32), -448, 448)
+    mine = np.array([synth.e4m3(float(t)) for t in v], dtype=np.uint8)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(mine, ref)
+    assert synth.e4m3(1e9) == 0x7E and synth.e4m3(-1e9) == 0xFE  # saturation
+
+
+def test_generator_gaussian_exponent_histogram_matches_binade_probabilities():
+    """N(0,1)*16 cast with RNE: exponent field k collects |x| in
+    [0.96875 * 2^(k-7), 0.96875 * 2^(k-6)) (the rounding midpoints)."""
+    spec = synth.single_normal_1k().tensors[0]
+    x = spec.generate()
+    hist = np.bincount((x >> 3) & 15, minlength=16).astype(np.float64)
+    n = x.size
+    phi = lambda t: 0.5 * (1 + math.erf(t / math.sqrt(2)))  # noqa: E731
+    p_abs_below = lambda t: 2 * phi(t / 16.0) - 1  # noqa: E731
+    edges = [0.0, 0.9375 * 2 ** -6] + [0.96875 * 2 ** (k - 6) for k in range(1, 15)] + [math.inf]
+    probs = [(1.0 if b == math.inf else p_abs_below(b)) - p_abs_below(a) for a, b in zip(edges[:-1], edges[1:])]
+    for k in range(16):
+        exp = probs[k] * n
+        assert abs(hist[k] - exp) <= 5 * math.sqrt(exp + 1) + 1, (k, hist[k], exp)
+
+
+def test_generator_alpha_two_is_gaussian_with_variance_two():
+    z = synth.sas_raw(synth.SEED_BASE, 400_000, 2.0)
+    assert abs(z.mean()) < 0.02 and abs(z.var() - 2.0) < 0.03
+    g = synth.normal_raw(synth.SEED_BASE, 400_000)
+    assert abs(g.mean()) < 0.01 and abs(g.var() - 1.0) < 0.015
+
+
+def test_generator_heavy_tail_index():
+    """P(|X| > t) ~ C t^-alpha for alpha < 2: the log-log slope of the tail."""
+    z = np.abs(synth.sas_raw(synth.SEED_BASE + 1, 1_000_000, 1.5))
+    t1, t2 = 20.0, 80.0
+    s = math.log((z > t2).mean() / (z > t1).mean()) / math.log(t2 / t1)
+    assert abs(s + 1.5) < 0.12
+
+
+def test_exponent_entropy_in_the_pages_range_for_gaussian():
+    """alpha = 2 weights: about 2.55-2.75 bits of exponent entropy (p1 §2.2)."""
+    x = synth.alpha_sweep_point(2.0, 448.0).tensors[0].generate(count=1 << 21)
+    H = _entropy_bits(np.bincount((x >> 3) & 15, minlength=16))
+    assert 2.4 < H < 2.8
