@@ -23,7 +23,9 @@
  *  - code stream: little-endian 32-bit words, bit i of the stream is bit
  *    31 - (i mod 32) of word i / 32 (MSB first within a word).
  *  - chunk c = stream bits [8Cc, 8C(c+1)); gap_c = first code start at or
- *    after 8Cc minus 8Cc (0 if none), 4 bits per chunk (p1 §3.2.1 gap[tid]).
+ *    after 8Cc minus 8Cc, 4 bits per chunk (p1 §3.2.1 gap[tid]).  The end of
+ *    the stream (bit code_bits) counts as a start, so a chunk that begins
+ *    inside the last code points past it; chunks beyond the end hold 0.
  *  - group g = T chunks; off[g] = number of codes starting before bit 8CTg.
  *  - nibbles: weight i lives in byte 4(i/8) + (i mod 4), low half if
  *    i mod 8 < 4, high half otherwise.
@@ -325,9 +327,10 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
   uint64_t chunk_bits = 8ull * C, chunks = L.groups * T;
   uint64_t next_chunk = 0;  /* first chunk whose gap is not yet known */
   uint64_t pos = 0;
-  for (uint64_t i = 0; i < n; ++i) {
+  for (uint64_t i = 0; i <= n; ++i) {
     /* every chunk that starts at or before this code's start, and after the
-     * previous code's start, has this code as its first code */
+     * previous code's start, has this code as its first code; i == n is the
+     * end of the stream */
     while (next_chunk < chunks && next_chunk * chunk_bits <= pos) {
       uint64_t gap = pos - next_chunk * chunk_bits;
       if (gap > 15) return -4;
@@ -336,13 +339,14 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
       if (next_chunk % T == 0) wr64(offs + 8 * (next_chunk / T), i);
       next_chunk += 1;
     }
+    if (i == n) break;
     int e = oracle_exponent(x[i]);
     for (int b = len[e] - 1; b >= 0; --b) {
       if ((code[e] >> b) & 1u) set_bit(stream, pos);
       pos += 1;
     }
   }
-  /* chunks past the last code start keep gap 0; their groups start at n */
+  /* chunks wholly past the end keep gap 0; their groups start at n */
   for (; next_chunk < chunks; ++next_chunk)
     if (next_chunk % T == 0) wr64(offs + 8 * (next_chunk / T), n);
   wr64(offs + 8 * L.groups, n);
@@ -407,16 +411,18 @@ int oracle_check_index(const uint8_t* blob, uint64_t size) {
       if (rd32(blob + L.lut_off + 4 * p) != oracle_lut_entry(len, p)) return 1;
   const uint8_t* stream = blob + L.stream_off;
   uint64_t chunk_bits = 8ull * L.C, chunks = L.groups * L.T, c = 0, pos = 0;
-  for (uint64_t i = 0; i <= L.n; ++i) {
-    uint64_t start = i < L.n ? pos : UINT64_MAX; /* virtual start past the end */
+  for (uint64_t i = 0; i <= L.n + 1; ++i) {
+    /* code starts, then the end of the stream, then a start past every chunk */
+    uint64_t start = i < L.n ? pos : (i == L.n ? L.code_bits : UINT64_MAX);
     while (c < chunks && c * chunk_bits <= start) {
-      uint32_t want = i < L.n ? (uint32_t)(start - c * chunk_bits) : 0;
+      uint32_t want = i <= L.n ? (uint32_t)(start - c * chunk_bits) : 0;
       uint32_t got = (rd32(blob + L.gaps_off + 4 * (c / 8)) >> (4 * (c % 8))) & 15u;
       if (got != want) return 2;
-      if (c % L.T == 0 && rd64(blob + L.groups_off + 8 * (c / L.T)) != i) return 3;
+      uint64_t first = i < L.n ? i : L.n;
+      if (c % L.T == 0 && rd64(blob + L.groups_off + 8 * (c / L.T)) != first) return 3;
       c += 1;
     }
-    if (i == L.n) break;
+    if (i >= L.n) continue;
     int used = 0;
     if (match_code(len, code, stream_bit, stream, pos, L.code_bits - pos, &used) < 0) return 4;
     pos += (uint64_t)used;

@@ -402,3 +402,31 @@ def test_exponent_entropy_in_the_pages_range_for_gaussian():
     x = synth.alpha_sweep_point(2.0, 448.0).tensors[0].generate(count=1 << 21)
     H = _entropy_bits(np.bincount((x >> 3) & 15, minlength=16))
     assert 2.4 < H < 2.8
+
+
+def test_gaps_and_offsets_from_code_start_positions():
+    """gap_c = (first code start >= 8Cc, the stream end counting as a start) - 8Cc,
+    off[g] = number of codes starting before bit 8CTg; recomputed here from the
+    cumulative code lengths with numpy."""
+    r = _rng(31)
+    vals = np.array([0x38, 0x40, 0x00, 0x30, 0x41, 0xB8], np.uint8)
+    for trial in range(300):
+        n = int(r.integers(1, 400))
+        x = r.choice(vals, size=n, p=[.5, .2, .1, .1, .05, .05])
+        C, T = int(r.choice([4, 8])), int(r.integers(1, 5))
+        blob = oracle.encode(x, chunk_bytes=C, group_chunks=T)
+        hd = oracle.blob_header(blob)
+        lens = hd["lengths"][(x >> 3) & 15].astype(np.int64)
+        starts = np.concatenate([[0], np.cumsum(lens)])  # last entry = code_bits
+        assert starts[-1] == hd["code_bits"]
+        chunks = hd["n_groups"] * T
+        gw = blob[hd["gaps_off"]:hd["gaps_off"] + 4 * ((chunks + 7) // 8)].view("<u4")
+        for c in range(chunks):
+            b0 = 8 * C * c
+            got = (int(gw[c // 8]) >> (4 * (c % 8))) & 15
+            want = int(starts[np.searchsorted(starts, b0)] - b0) if b0 <= starts[-1] else 0
+            assert got == want, (trial, c)
+        offs = blob[hd["groups_off"]:hd["groups_off"] + 8 * (hd["n_groups"] + 1)].view("<u8")
+        for g in range(hd["n_groups"] + 1):
+            want = min(int(np.searchsorted(starts[:-1], 8 * C * T * g)), n)
+            assert int(offs[g]) == want
