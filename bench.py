@@ -1,0 +1,447 @@
+#!/usr/bin/env python3
+"""ECF8 decode benchmark.
+
+One step = one batched decode launch over every tensor of the workload (the
+whole hot path: table load, chunk walk, scan, compaction, assembly, store),
+inputs resident in HBM.  Default workload: the seven projections of one
+Llama-3-8B decoder layer in FP8 E4M3 (q/o 4096x4096, k/v 1024x4096, gate/up
+14336x4096, down 4096x14336), weights symmetric alpha-stable alpha=1.8 scaled
+to max|w| = 448, one codebook per tensor: 218,103,808 bytes of FP8 out.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun): every rank decodes its own copy of the layer (weak
+scaling; the decode has no exchange step), time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ecf8_synth as synth  # noqa: E402
+
+METRIC = "ECF8 decode GB/s (FP8 out) and % of HBM roofline on 1 B200; compression ratio"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SRC = os.path.join(ROOT, "lossless_fp8_weight_b200", "csrc", "ecf8_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
+def workload_by_name(name: str) -> synth.Workload:
+    if name == "llama3_8b_layer":
+        return synth.llama3_8b_layer()
+    if name == "single_1k":
+        return synth.single_normal_1k()
+    if name.startswith("sweep_"):  # sweep_<alpha>_<max>
+        _, a, m = name.split("_")
+        return synth.alpha_sweep_point(float(a), float(m))
+    if name.startswith("moe"):
+        k = int(name[3:] or 256)
+        return synth.moe_experts(k)
+    if name.startswith("llama3_70b_layer"):
+        return synth.llama3_70b_layer(int(name[len("llama3_70b_layer"):] or 0))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def entropy_bits(hist) -> float:
+    h = np.asarray(hist, dtype=np.float64)
+    p = h[h > 0] / h.sum()
+    return float(-(p * np.log2(p)).sum())
+
+
+def prepare(workload: synth.Workload, L):
+    """Generate and encode every tensor on the host (not timed)."""
+    blobs, xs, stats = [], [], []
+    for t in workload.tensors:
+        x = t.generate()
+        hist = L.histogram(x)
+        cb = L.build_codebook(hist)
+        blob = L.encode(x, codebook=cb)
+        info = L.blob_info(blob)
+        lens = info.lengths.astype(np.float64)
+        stats.append({"n": int(x.size), "blob": int(blob.size), "hist": hist,
+                      "code_bits": int(info.code_bits), "le6": float(hist[lens <= 6].sum()) / x.size,
+                      "max_len": int(info.max_len)})
+        blobs.append(blob)
+        xs.append(x)
+    return blobs, xs, stats
+
+
+def compression_summary(stats):
+    n = sum(s["n"] for s in stats)
+    blob = sum(s["blob"] for s in stats)
+    hist = sum(s["hist"].astype(np.float64) for s in stats)
+    return {
+        "n_bytes": n,
+        "compressed_bytes": blob,
+        "ratio": round(n / blob, 4),
+        "savings_pct": round(100 * (1 - blob / n), 2),
+        "exponent_entropy_bits": round(entropy_bits(hist), 4),
+        "mean_code_bits": round(sum(s["code_bits"] for s in stats) / n, 4),
+        "codes_le6_bits_frac": round(sum(s["le6"] * s["n"] for s in stats) / n, 5),
+        "max_code_bits": max(s["max_len"] for s in stats),
+    }
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sha() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source and this workload."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        if rec.get("kernel_sha") == kernel_sha() and rec.get("workload") == workload_name:
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons, power = [], [], set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def oracle_cpu_baseline(blobs, xs, budget_s: float = 12.0):
+    """Time the bit-serial oracle decoding tensors of the workload on host
+    threads (one tensor per thread) for a bounded sample."""
+    import oracle
+    cores = min(len(blobs), os.cpu_count() or 1)
+    order = sorted(range(len(blobs)), key=lambda i: xs[i].size)
+    # a bounded sample: smallest tensors first until the estimated work fits the budget
+    est_rate = 12e6  # weights/s per core, for sizing only
+    picked, work = [], 0.0
+    for i in order:
+        if picked and (work + xs[i].size / est_rate) / cores > budget_s:
+            break
+        picked.append(i)
+        work += xs[i].size / est_rate
+    outs = {i: np.empty(xs[i].size, np.uint8) for i in picked}
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        rcs = list(ex.map(lambda i: oracle.decode_into(blobs[i], outs[i]), picked))
+    dt = time.perf_counter() - t0
+    assert all(rc == 0 for rc in rcs)
+    for i in picked:
+        assert np.array_equal(outs[i], xs[i])
+    n = sum(xs[i].size for i in picked)
+    return {"value": round(n / dt / 1e9, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(picked)} of {len(blobs)} tensors ({n} weights), one tensor per thread, "
+                      f"{dt:.2f} s"}
+
+
+def run_reference(args, workload):
+    """The oracle as the reference arm: host cores, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    L = load_library(build_only=True)
+    sample = int(args.ref_sample)
+    blobs, xs = [], []
+    for t in workload.tensors:
+        x = t.generate(count=min(sample, t.n), scale=t.scale() if t.dist == "sas" else None)
+        xs.append(x)
+        blobs.append(L.encode(x))
+    cores = min(len(blobs), os.cpu_count() or 1)
+    outs = [np.empty(x.size, np.uint8) for x in xs]
+
+    def step():
+        with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+            rcs = list(ex.map(lambda i: oracle.decode_into(blobs[i], outs[i]), range(len(blobs))))
+        assert all(rc == 0 for rc in rcs)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    for x, o in zip(xs, outs):
+        assert np.array_equal(x, o)
+    n = sum(x.size for x in xs) * args.steps
+    value = n / dt / 1e9
+    summ = compression_summary([{"n": x.size, "blob": b.size, "hist": L.histogram(x),
+                                 "code_bits": int(L.blob_info(b).code_bits), "le6": 0.0,
+                                 "max_len": int(L.blob_info(b).max_len)} for x, b in zip(xs, blobs)])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": workload.name, "tensors": len(workload.tensors),
+                   "sample_weights_per_tensor": sample, "ratio_of_sample": summ["ratio"]},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {sample} weights of each of the {len(xs)} tensors, "
+                                   "one tensor per thread, per step"},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (timing is the
+    slowest rank's); a no-op without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def load_library(build_only=False):
+    from lossless_fp8_weight_b200 import _build
+    _build.build()
+    import lossless_fp8_weight_b200 as L
+    return L
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_layer")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--ref-sample", type=int, default=1 << 21)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    workload = workload_by_name(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, workload)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    L = load_library()
+
+    blobs, xs, stats = prepare(workload, L)
+    infos = [L.blob_info(b) for b in blobs]
+    n_total = sum(i.n for i in infos)
+    blob_total = sum(int(b.size) for b in blobs)
+
+    dev = torch.device("cuda", local)
+    # all blobs in one allocation, each at a 256-byte boundary
+    offs, o = [], 0
+    for b in blobs:
+        offs.append(o)
+        o += (b.size + 255) // 256 * 256
+    d_blobs = torch.empty(o, dtype=torch.uint8, device=dev)
+    for b, off in zip(blobs, offs):
+        d_blobs[off:off + b.size].copy_(torch.from_numpy(b))
+    out_offs, o = [], 0
+    for i in infos:
+        out_offs.append(o)
+        o += (i.n + 255) // 256 * 256
+    d_out = torch.empty(o, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_bytes = max(L.batched_workspace_size(len(infos)), 16)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    items = [L.BatchItem(i, int(d_blobs.data_ptr()) + bo, int(d_out.data_ptr()) + oo)
+             for i, bo, oo in zip(infos, offs, out_offs)]
+    batch = L.make_batch(items)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        L.decode_batched(batch, workspace=ws, status=status, stream=stream)
+
+    # correctness of the timed configuration: bit-exact against the source bytes
+    step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"decode status {int(status.item())}"
+    host_out = d_out.cpu().numpy()
+    for x, oo in zip(xs, out_offs):
+        if not np.array_equal(host_out[oo:oo + x.size], x):
+            raise SystemExit("decode mismatch in the benchmark configuration")
+    del host_out
+
+    # warm-up (and a >= 1 s pre-roll under the clock sampler)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0
+    w = 0
+    while w < args.warmup or time.perf_counter() < t_end:
+        step()
+        w += 1
+        if w % 50 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches0 = L.launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = L.launch_count() - launches0
+    clk = clocks.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    elapsed_ms, per_launch_ms = max_over_ranks([elapsed_ms, per_launch_ms], dev)
+    if world > 1:
+        dist.barrier()
+    assert int(status.item()) == 0
+
+    # end to end through the same call: pinned host blob -> device, decode,
+    # device -> pinned host output, every step
+    h_blob = torch.empty(d_blobs.numel(), dtype=torch.uint8, pin_memory=True)
+    for b, off in zip(blobs, offs):
+        h_blob[off:off + b.size].copy_(torch.from_numpy(b))
+    h_out = torch.empty(d_out.numel(), dtype=torch.uint8, pin_memory=True)
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+
+    def e2e_step():
+        d_blobs.copy_(h_blob, non_blocking=True)
+        step()
+        h_out.copy_(d_out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
+    out_np = h_out.numpy()
+    for x, oo in zip(xs, out_offs):
+        assert np.array_equal(out_np[oo:oo + x.size], x)
+
+    value = n_total * args.steps * world / (elapsed_ms / 1e3) / 1e9
+    e2e_value = n_total * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    alg_bytes = blob_total + n_total  # compressed bytes read + FP8 bytes written
+    achieved = alg_bytes / (per_launch_ms / 1e3) / 1e9
+    traffic = recorded_traffic(workload.name)
+    comp = compression_summary(stats)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_cpu_baseline(blobs, xs)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": workload.name, "description": workload.description,
+                       "tensors": len(workload.tensors), "batched_launch": True,
+                       "chunk_bytes": int(infos[0].chunk_bytes), "group_chunks": int(infos[0].group_chunks),
+                       "l2": "inputs+outputs larger than L2 (no flush)"
+                             if alg_bytes > L2_BYTES else "fits in L2 (no flush)",
+                       **comp},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": alg_bytes,
+                         "launch_ms": round(per_launch_ms, 5)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 3), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(blob_total), "d2h_bytes_per_step": int(n_total),
+                    "steps": e2e_steps},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * ecf8.h -- C ABI of the ECF8 (Exponent-Concentrated FP8) lossless codec for
+ * FP8 E4M3 weight tensors: host-side encoder and sm_100a GPU decoder.
+ *
+ * Method ("To Compress or Not? Pushing the Frontier of Lossless GenAI Model
+ * Weights Compression with Exponent Concentration", arXiv 2510.02676,
+ * abstract; ECF8 walkthrough "ECF8 浮点数压缩技术" §3.1-§3.2): the 4-bit exponent
+ * field of every E4M3 weight is coded with a per-tensor canonical Huffman
+ * code of at most 16 bits, sign and mantissa are kept raw as a nibble array,
+ * and decoding reproduces every original byte exactly.
+ *
+ * Conventions for every call:
+ *  - Return value: ECF8_OK (0) or a negative ECF8_ERR_* code; ecf8_strerror
+ *    names it.  No call throws, aborts or prints.
+ *  - The caller owns every buffer, host and device.  The library keeps no
+ *    state between calls except per-device kernel attributes set once, and a
+ *    launch counter; it allocates no device memory.
+ *  - "host" pointers are ordinary CPU memory; "device" pointers are CUDA
+ *    global memory of the current device and must be 16-byte aligned.
+ *  - Decode calls are asynchronous on the given stream.  Argument and header
+ *    errors are returned before anything is enqueued.  Corrupt data found by
+ *    the kernel is reported by OR-ing ECF8_STATUS_* bits into *d_status
+ *    (device int32, nullable), which the caller reads after synchronising.
+ *    The kernels never write outside [d_out, d_out + n) and never wait.
+ *
+ * Blob layout (version 1, all fields little-endian; the on-disk and in-HBM
+ * form of one compressed tensor):
+ *   header, 128 bytes:
+ *     0 u32 magic 0x38464345 ("ECF8")   4 u32 version = 1
+ *     8 u64 n (weights)                16 u64 code_bits (stream length in bits)
+ *    24 u32 chunk_bytes C              28 u32 group_chunks T
+ *    32 u32 n_groups G                 36 u32 lut_bits = 12
+ *    40 u32 max code length            44 u32 header bytes = 128
+ *    48 u64 offset of decode table     56 u64 offset of gaps
+ *    64 u64 offset of group offsets    72 u64 offset of code stream
+ *    80 u64 offset of nibbles          88 u64 blob bytes
+ *    96 u8[16] code length per exponent value (0 = absent)   112 u8[16] zero
+ *   sections, each at a multiple of 256 bytes, in this order:
+ *     decode table  4096 u32 (absent when n = 0).  Entry for a 12-bit window:
+ *                   bits 0-3 bits used, 4-6 codes (0..6), 8+4j exponent j,
+ *                   the greedy decode of the codes lying wholly in the window.
+ *     gaps          4 bits per chunk, chunk c in bits 4(c%8) of u32 word c/8;
+ *                   offset of the first code start at or after the chunk start
+ *                   (the stream end counts as a start), 0 past the end.
+ *     group offsets G+1 u64: number of codes starting before bit 8*C*T*g.
+ *     code stream   G*T*C bytes + 16 zero bytes; u32 words, stream bit i is
+ *                   bit 31-(i%32) of word i/32.
+ *     nibbles       ceil(n/32)*16 bytes; weight i's (sign<<3 | mantissa) in
+ *                   byte 4(i/8)+(i%4), low half if i%8 < 4 else high half.
+ */
+#ifndef ECF8_H_
+#define ECF8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h> /* cudaStream_t */
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ECF8_ABI_VERSION 1
+
+/* return codes */
+#define ECF8_OK 0
+#define ECF8_ERR_ARG (-1)         /* null pointer, bad size or parameter */
+#define ECF8_ERR_FORMAT (-2)      /* blob header or layout inconsistent */
+#define ECF8_ERR_CAPACITY (-3)    /* destination buffer too small */
+#define ECF8_ERR_CODEBOOK (-4)    /* invalid code lengths, or an exponent with no code */
+#define ECF8_ERR_ALIGN (-5)       /* device pointer not 16-byte aligned */
+#define ECF8_ERR_UNSUPPORTED (-6) /* layout the GPU kernels do not implement */
+#define ECF8_ERR_CUDA (-7)        /* a CUDA runtime call failed */
+#define ECF8_ERR_WORKSPACE (-8)   /* workspace null or too small */
+
+/* bits OR-ed into *d_status by the decode kernels */
+#define ECF8_STATUS_COUNT_MISMATCH 1 /* codes decoded in a group != its offset delta */
+#define ECF8_STATUS_BAD_CODE 2       /* bits that match no code */
+#define ECF8_STATUS_BAD_OFFSETS 4    /* group offsets not monotone or past n */
+
+/* A canonical Huffman code over the 16 exponent values. */
+typedef struct ecf8_codebook {
+  uint8_t len[16];   /* code length in bits, 0 = value absent */
+  uint16_t code[16]; /* canonical code, right-aligned, valid where len > 0 */
+  uint32_t max_len;  /* longest length present */
+  uint32_t n_symbols;
+} ecf8_codebook;
+
+/* Header of one blob, as read on the host by ecf8_blob_info.  Decode calls
+ * take it so that they never read the device blob back. */
+typedef struct ecf8_info {
+  uint64_t n;
+  uint64_t code_bits;
+  uint64_t blob_bytes;
+  uint64_t lut_off, gaps_off, groups_off, stream_off, nibbles_off;
+  uint32_t chunk_bytes;
+  uint32_t group_chunks;
+  uint32_t n_groups;
+  uint32_t lut_bits;
+  uint32_t max_len;
+  uint8_t len[16];
+} ecf8_info;
+
+/* One tensor of a batched decode. */
+typedef struct ecf8_tensor {
+  const ecf8_info* info; /* host */
+  const void* d_blob;    /* device, 16-byte aligned, info->blob_bytes long */
+  uint8_t* d_out;        /* device, 16-byte aligned, info->n bytes */
+} ecf8_tensor;
+
+/* Exponent histogram of n E4M3 bytes (ECF8 walkthrough §3.1.1 step 1,
+ * §5.1 collect_exp_stats).  host in, host out. */
+int ecf8_histogram(const uint8_t* fp8, size_t n, uint64_t hist[16]);
+
+/* Optimal prefix code of at most max_len bits (1..16) for a histogram (§3.1.1
+ * steps 2-3, build_huffman).  Huffman with ties broken by (weight, node id),
+ * leaves numbered by value and merged nodes 16, 17, ...; when that tree is
+ * deeper than max_len, package-merge.  A single present value gets a 1-bit
+ * code.  ECF8_ERR_CODEBOOK when 2^max_len < number of present values. */
+int ecf8_build_codebook(const uint64_t hist[16], uint32_t max_len, ecf8_codebook* out);
+
+/* Exact blob size for n weights with histogram hist under cb.  host. */
+int ecf8_encoded_size(const uint64_t hist[16], size_t n, const ecf8_codebook* cb,
+                      uint32_t chunk_bytes, uint32_t group_chunks, size_t* out_bytes);
+
+/* Encode n E4M3 bytes into blob (host, capacity cap).  chunk_bytes is the
+ * stream slice of one decoder thread (multiple of 4), group_chunks the chunks
+ * that share one group offset.  ECF8_ERR_CODEBOOK if a present exponent has
+ * no code; ECF8_ERR_CAPACITY if cap is short.  *blob_bytes gets the size. */
+int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t chunk_bytes,
+                uint32_t group_chunks, void* blob, size_t cap, size_t* blob_bytes);
+
+/* Parse and check a host copy of a blob: magic, version, layout, lengths
+ * (Kraft sum <= 1) and the decode table against the lengths. */
+int ecf8_blob_info(const void* blob, size_t size, ecf8_info* out);
+
+/* 1 if the GPU kernels implement (chunk_bytes, group_chunks), else 0. */
+int ecf8_layout_supported(uint32_t chunk_bytes, uint32_t group_chunks);
+
+/* Decode one tensor on the GPU (§3.2.1): d_blob (device copy of the blob
+ * described by info) -> d_out, n must equal info->n.  One kernel launch on
+ * stream s; no launch when n = 0. */
+int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_t n,
+                int32_t* d_status, cudaStream_t s);
+
+/* Batches of at most this many tensors need no workspace. */
+#define ECF8_BATCH_INLINE_MAX 64
+
+/* Bytes of device workspace ecf8_decode_batched needs for count tensors
+ * (0 when count <= ECF8_BATCH_INLINE_MAX). */
+size_t ecf8_batched_workspace_size(int count);
+
+/* Decode count tensors in ONE kernel launch (batching across tensors as in
+ * the DFloat11 article's block-level batching, "Transformer块级批处理").  All
+ * tensors must share chunk_bytes and group_chunks.  Up to
+ * ECF8_BATCH_INLINE_MAX tensors travel in the launch's parameter block and
+ * d_workspace may be NULL.  Larger batches copy a descriptor table host->device
+ * into d_workspace (device, 16-byte aligned) on stream s before the launch;
+ * the workspace must not be touched by other streams until the decode ends. */
+int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
+                        int32_t* d_status, cudaStream_t s);
+
+/* Number of decode kernels this library has launched in this process. */
+uint64_t ecf8_launch_count(void);
+
+const char* ecf8_strerror(int code);
+int ecf8_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ECF8_H_ */

@@ -1,0 +1,213 @@
+"""ECF8 lossless FP8 E4M3 weight codec: Python binding of libecf8.
+
+Thin ctypes layer over the C ABI in ``include/ecf8.h``: it marshals arguments
+and nothing else.  Encoding runs in the library's host code; every step of
+decoding runs in its sm_100a kernels.  PyTorch is used only to hand over
+device pointers and the current CUDA stream.  There is no CPU fallback: if
+``libecf8.so`` is missing, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libecf8.so")
+
+if not os.path.exists(_SO):
+    raise ImportError(
+        f"{_SO} is missing: build it with `python -m lossless_fp8_weight_b200._build` "
+        "(or __graft_entry__.build()); the decoder has no CPU fallback")
+
+_lib = ctypes.CDLL(_SO)
+
+OK = 0
+ERRORS = {-1: "ARG", -2: "FORMAT", -3: "CAPACITY", -4: "CODEBOOK", -5: "ALIGN", -6: "UNSUPPORTED", -7: "CUDA",
+          -8: "WORKSPACE"}
+STATUS_COUNT_MISMATCH = 1
+STATUS_BAD_CODE = 2
+STATUS_BAD_OFFSETS = 4
+BATCH_INLINE_MAX = 64
+DEFAULT_CHUNK_BYTES = 32
+DEFAULT_GROUP_CHUNKS = 128
+
+
+class Codebook(ctypes.Structure):
+    _fields_ = [("len", ctypes.c_uint8 * 16), ("code", ctypes.c_uint16 * 16), ("max_len", ctypes.c_uint32),
+                ("n_symbols", ctypes.c_uint32)]
+
+    @property
+    def lengths(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.len), dtype=np.uint8).copy()
+
+
+class Info(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_uint64), ("code_bits", ctypes.c_uint64), ("blob_bytes", ctypes.c_uint64),
+                ("lut_off", ctypes.c_uint64), ("gaps_off", ctypes.c_uint64), ("groups_off", ctypes.c_uint64),
+                ("stream_off", ctypes.c_uint64), ("nibbles_off", ctypes.c_uint64),
+                ("chunk_bytes", ctypes.c_uint32), ("group_chunks", ctypes.c_uint32), ("n_groups", ctypes.c_uint32),
+                ("lut_bits", ctypes.c_uint32), ("max_len", ctypes.c_uint32), ("len", ctypes.c_uint8 * 16)]
+
+    @property
+    def lengths(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.len), dtype=np.uint8).copy()
+
+    @property
+    def ratio(self) -> float:
+        return self.n / self.blob_bytes if self.blob_bytes else 0.0
+
+
+class Tensor(ctypes.Structure):
+    _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("d_out", ctypes.c_void_p)]
+
+
+_p, _sz, _u32, _i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_int
+_lib.ecf8_histogram.argtypes = [_p, _sz, _p]
+_lib.ecf8_build_codebook.argtypes = [_p, _u32, ctypes.POINTER(Codebook)]
+_lib.ecf8_encoded_size.argtypes = [_p, _sz, ctypes.POINTER(Codebook), _u32, _u32, ctypes.POINTER(_sz)]
+_lib.ecf8_encode.argtypes = [_p, _sz, ctypes.POINTER(Codebook), _u32, _u32, _p, _sz, ctypes.POINTER(_sz)]
+_lib.ecf8_blob_info.argtypes = [_p, _sz, ctypes.POINTER(Info)]
+_lib.ecf8_layout_supported.argtypes = [_u32, _u32]
+_lib.ecf8_decode.argtypes = [ctypes.POINTER(Info), _p, _p, _sz, _p, _p]
+_lib.ecf8_batched_workspace_size.argtypes = [_i32]
+_lib.ecf8_batched_workspace_size.restype = _sz
+_lib.ecf8_decode_batched.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p]
+_lib.ecf8_launch_count.restype = ctypes.c_uint64
+_lib.ecf8_strerror.restype = ctypes.c_char_p
+_lib.ecf8_strerror.argtypes = [_i32]
+
+
+class Ecf8Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {_lib.ecf8_strerror(code).decode()} ({ERRORS.get(code, code)})")
+        self.code = code
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != OK:
+        raise Ecf8Error(rc, what)
+
+
+def library_path() -> str:
+    return _SO
+
+
+def launch_count() -> int:
+    """Decode kernels launched by this process so far."""
+    return int(_lib.ecf8_launch_count())
+
+
+def _host_u8(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # a CPU torch tensor
+        x = x.detach().contiguous().view(-1).numpy()
+    a = np.ascontiguousarray(np.asarray(x).reshape(-1))
+    if a.dtype != np.uint8:
+        a = a.view(np.uint8)
+    return a
+
+
+def histogram(fp8) -> np.ndarray:
+    x = _host_u8(fp8)
+    h = np.zeros(16, dtype=np.uint64)
+    _check(_lib.ecf8_histogram(x.ctypes.data, x.size, h.ctypes.data), "ecf8_histogram")
+    return h
+
+
+def build_codebook(hist, max_len: int = 16) -> Codebook:
+    h = np.ascontiguousarray(np.asarray(hist, dtype=np.uint64))
+    cb = Codebook()
+    _check(_lib.ecf8_build_codebook(h.ctypes.data, max_len, ctypes.byref(cb)), "ecf8_build_codebook")
+    return cb
+
+
+def encode(fp8, codebook: Optional[Codebook] = None, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
+           group_chunks: int = DEFAULT_GROUP_CHUNKS, max_len: int = 16) -> np.ndarray:
+    """Compress E4M3 bytes (numpy uint8 / float8 view, or CPU tensor) into a blob."""
+    x = _host_u8(fp8)
+    h = histogram(x)
+    cb = codebook if codebook is not None else build_codebook(h, max_len)
+    size = ctypes.c_size_t(0)
+    _check(_lib.ecf8_encoded_size(h.ctypes.data, x.size, ctypes.byref(cb), chunk_bytes, group_chunks,
+                                  ctypes.byref(size)), "ecf8_encoded_size")
+    blob = np.empty(size.value, dtype=np.uint8)
+    got = ctypes.c_size_t(0)
+    _check(_lib.ecf8_encode(x.ctypes.data, x.size, ctypes.byref(cb), chunk_bytes, group_chunks, blob.ctypes.data,
+                            blob.size, ctypes.byref(got)), "ecf8_encode")
+    assert got.value == blob.size
+    return blob
+
+
+def blob_info(blob) -> Info:
+    b = _host_u8(blob)
+    info = Info()
+    _check(_lib.ecf8_blob_info(b.ctypes.data, b.size, ctypes.byref(info)), "ecf8_blob_info")
+    return info
+
+
+def layout_supported(chunk_bytes: int, group_chunks: int) -> bool:
+    return bool(_lib.ecf8_layout_supported(chunk_bytes, group_chunks))
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def decode(info: Info, d_blob, d_out, status=None, stream=None) -> None:
+    """Asynchronously decode one blob already in device memory into d_out
+    (torch uint8 CUDA tensors or raw device pointers) on ``stream``."""
+    _check(_lib.ecf8_decode(ctypes.byref(info), _ptr(d_blob), _ptr(d_out), info.n, _ptr(status),
+                            _stream(stream)), "ecf8_decode")
+
+
+def batched_workspace_size(count: int) -> int:
+    return int(_lib.ecf8_batched_workspace_size(count))
+
+
+@dataclass
+class BatchItem:
+    info: Info
+    d_blob: object
+    d_out: object
+
+
+def make_batch(items: Sequence[BatchItem]):
+    """The ctypes array a batched decode takes; keep it alive while reused."""
+    arr = (Tensor * len(items))()
+    keep = []
+    for i, it in enumerate(items):
+        keep.append(it.info)
+        arr[i].info = ctypes.pointer(it.info)
+        arr[i].d_blob = _ptr(it.d_blob)
+        arr[i].d_out = _ptr(it.d_out)
+    return arr, keep
+
+
+def decode_batched(items, workspace=None, status=None, stream=None) -> None:
+    """Decode several blobs in one kernel launch.  ``items`` is a list of
+    BatchItem or the pair returned by make_batch."""
+    if isinstance(items, tuple):
+        arr = items[0]
+    else:
+        arr, _keep = make_batch(items)
+    ws = _ptr(workspace)
+    ws_bytes = int(workspace.numel() * workspace.element_size()) if workspace is not None and not isinstance(
+        workspace, int) else 0
+    _check(_lib.ecf8_decode_batched(arr, len(arr), ws, ws_bytes, _ptr(status), _stream(stream)),
+           "ecf8_decode_batched")

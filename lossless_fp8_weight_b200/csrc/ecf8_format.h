@@ -1,0 +1,74 @@
+// Library-internal constants and layout arithmetic for the ECF8 blob (version 1),
+// shared by the host encoder (ecf8_host.cpp) and the decode kernels
+// (ecf8_decode.cu).  The layout itself is documented in include/ecf8.h.
+#pragma once
+
+#include <stdint.h>
+
+#include "ecf8.h"
+
+namespace ecf8 {
+
+constexpr uint32_t kMagic = 0x38464345u;  // "ECF8"
+constexpr uint32_t kVersion = 1;
+constexpr uint32_t kHeaderBytes = 128;
+constexpr uint32_t kLutBits = 12;  // decode window
+constexpr uint32_t kLutEntries = 1u << kLutBits;
+constexpr uint32_t kLutMaxSyms = 6;  // codes per table entry
+constexpr uint32_t kSectionAlign = 256;
+
+struct Layout {
+  uint64_t n, code_bits, groups;
+  uint32_t C, T;
+  uint64_t lut_off, lut_bytes;
+  uint64_t gaps_off, gaps_bytes;
+  uint64_t groups_off, groups_bytes;
+  uint64_t stream_off, stream_bytes;
+  uint64_t nib_off, nib_bytes;
+  uint64_t total;
+};
+
+inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// Section sizes and offsets for n weights whose codes take code_bits bits.
+inline bool compute_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t T, Layout* L) {
+  if (C < 4 || C % 4 != 0 || T < 1) return false;
+  L->n = n;
+  L->code_bits = code_bits;
+  L->C = C;
+  L->T = T;
+  const uint64_t group_bits = 8ull * C * T;
+  L->groups = (code_bits + group_bits - 1) / group_bits;
+  if (L->groups > 0xFFFFFFFFull) return false;
+  const uint64_t chunks = L->groups * T;
+  L->lut_bytes = n ? 4ull * kLutEntries : 0;
+  L->gaps_bytes = align_up((chunks + 7) / 8 * 4, 16);
+  L->groups_bytes = 8 * (L->groups + 1);
+  L->stream_bytes = n ? chunks * C + 16 : 0;
+  L->nib_bytes = (n + 31) / 32 * 16;
+  L->lut_off = align_up(kHeaderBytes, kSectionAlign);
+  L->gaps_off = align_up(L->lut_off + L->lut_bytes, kSectionAlign);
+  L->groups_off = align_up(L->gaps_off + L->gaps_bytes, kSectionAlign);
+  L->stream_off = align_up(L->groups_off + L->groups_bytes, kSectionAlign);
+  L->nib_off = align_up(L->stream_off + L->stream_bytes, kSectionAlign);
+  L->total = L->nib_off + L->nib_bytes;
+  return true;
+}
+
+// What a decode kernel needs to know about one tensor, with device pointers
+// already resolved into the blob's sections.
+struct alignas(16) DevTensor {
+  const uint32_t* lut;
+  const uint32_t* gaps;
+  const uint64_t* groups;
+  const uint32_t* stream;
+  const void* nibbles;  // 16-byte aligned
+  uint8_t* out;
+  uint64_t n;
+  uint64_t code_bits;
+  uint32_t n_groups;
+  uint32_t group_base;  // batched: groups of all earlier tensors in the launch
+  uint8_t len[16];
+};
+
+}  // namespace ecf8
