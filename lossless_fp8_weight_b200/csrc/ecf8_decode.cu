@@ -47,6 +47,8 @@ struct Shape {
   static constexpr int kMaxCodes = 8 * C * T;   // per group
   static constexpr int kStageWords = T * C + 8; // staged exponents, +32 for alignment
   static constexpr int kWarps = T / 32;
+  static constexpr int kNB = 8;          // nibble blocks a thread prefetches in registers
+  static constexpr int kMinBlocks = 4;   // CTAs per SM the smem budget allows
   // shared memory carve-up, in 32-bit words
   static constexpr int kLutOff = 0;
   static constexpr int kPrivOff = kLutOff + (int)kLutEntries;
@@ -184,62 +186,112 @@ __device__ __forceinline__ void step_single(Walker& w, const uint32_t* lut, cons
   w.pos += len;
 }
 
+// ---------------------------------------------------------------- per group
+
+// What one thread fetches ahead for a group: its stream slice (+ the next
+// word, for a code that straddles the slice end), the raw gap word, and the
+// group's two offsets.  Kept raw so the loads stay in flight until used.
+template <int C>
+struct GroupIn {
+  uint32_t w[C / 4 + 1];
+  uint32_t gapw;
+  uint64_t off0, off1;
+};
+
 template <int C, int T>
-__device__ __forceinline__ void decode_group(const DevTensor& d, uint32_t g, uint32_t* sm, int32_t* status) {
+__device__ __forceinline__ void fetch_group(const DevTensor* dt, uint32_t local, GroupIn<C>& in) {
+  using S = Shape<C, T>;
+  const uint64_t chunk = (uint64_t)local * T + threadIdx.x;
+  const uint32_t* stream = dt->stream;
+  const uint4* cs = reinterpret_cast<const uint4*>(stream + chunk * S::kWords);
+#pragma unroll
+  for (int q = 0; q < S::kWords / 4; ++q) {
+    const uint4 v = __ldg(cs + q);
+    in.w[4 * q + 0] = v.x;
+    in.w[4 * q + 1] = v.y;
+    in.w[4 * q + 2] = v.z;
+    in.w[4 * q + 3] = v.w;
+  }
+  in.w[S::kWords] = __ldg(stream + (chunk + 1) * S::kWords);
+  in.gapw = __ldg(dt->gaps + (chunk >> 3));
+  in.off0 = __ldg(dt->groups + local);
+  in.off1 = __ldg(dt->groups + local + 1);
+}
+
+// K0: the tensor's decode table and canonical tables into shared memory.
+template <int C, int T>
+__device__ __forceinline__ void load_tables(const DevTensor* dt, uint32_t* lut, Canon* canon) {
+  const uint4* src = reinterpret_cast<const uint4*>(dt->lut);
+  uint4* dst = reinterpret_cast<uint4*>(lut);
+#pragma unroll 4
+  for (int i = threadIdx.x; i < (int)kLutEntries / 4; i += T) dst[i] = __ldg(src + i);
+  if (threadIdx.x == 0) build_canon(dt->len, canon);
+  __syncthreads();
+}
+
+// K4b + K5 for one 32-weight block: staged exponents + nibbles -> 32 bytes.
+__device__ __forceinline__ void store_block(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1, const uint4 ex,
+                                            const uint4 nb) {
+  uint32_t o[8];
+  assemble8(ex.x, nb.x, o[0], o[1]);
+  assemble8(ex.y, nb.y, o[2], o[3]);
+  assemble8(ex.z, nb.z, o[4], o[5]);
+  assemble8(ex.w, nb.w, o[6], o[7]);
+  uint8_t* dst = out + gpos;
+  if (gpos >= off0 && gpos + 32 <= off1) {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  } else {  // the group's ragged ends: bytes inside [off0, off1) only
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const uint64_t i = gpos + k;
+      if (i >= off0 && i < off1) dst[k] = (uint8_t)(o[k >> 2] >> (8 * (k & 3)));
+    }
+  }
+}
+
+template <int C, int T>
+__device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t local, const GroupIn<C>& in, uint32_t* sm,
+                                              int32_t* status) {
   using S = Shape<C, T>;
   uint32_t* lut = sm + S::kLutOff;
   uint32_t* priv = sm + S::kPrivOff;
   uint32_t* stage = sm + S::kStageOff;
   uint32_t* scan = sm + S::kScanOff;
-  Canon* canon = reinterpret_cast<Canon*>(sm + S::kCanonOff);
+  const Canon* canon = reinterpret_cast<const Canon*>(sm + S::kCanonOff);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const uint64_t n = dt->n;
+  const uint64_t off0 = in.off0, off1 = in.off1;
+  const bool offsets_ok = off0 <= off1 && off1 <= n && off1 - off0 <= (uint64_t)S::kMaxCodes;
 
-  // K0: decode table and canonical tables into shared memory
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(d.lut);
-    uint4* dst = reinterpret_cast<uint4*>(lut);
-#pragma unroll 4
-    for (int i = t; i < (int)kLutEntries / 4; i += T) dst[i] = __ldg(src + i);
-    if (t == 0) build_canon(d.len, canon);
-  }
-  const uint64_t off0 = __ldg(d.groups + g), off1 = __ldg(d.groups + g + 1);
-
-  // K1: this thread's chunk (+ the next word for a code that straddles the end)
-  const uint64_t chunk = (uint64_t)g * T + t;
-  const uint64_t bit0 = chunk * (8ull * C);
-  Walker w;
-  const uint64_t left = bit0 < d.code_bits ? d.code_bits - bit0 : 0;
-  w.end = left < 8ull * C ? (int)left : 8 * C;
-  const uint32_t gap = (__ldg(d.gaps + (chunk >> 3)) >> ((chunk & 7) * 4)) & 15u;
-  uint32_t word[S::kWords + 1];
-  {
-    const uint4* cs = reinterpret_cast<const uint4*>(d.stream + chunk * S::kWords);
+  // this group's nibbles: issued now, consumed after the walk
+  const uint32_t blocks = offsets_ok ? (uint32_t)(((off0 & 31) + (off1 - off0) + 31) >> 5) : 0;
+  const uint4* nib = reinterpret_cast<const uint4*>(dt->nibbles) + (off0 >> 5);
+  uint4 nv[S::kNB];
 #pragma unroll
-    for (int q = 0; q < S::kWords / 4; ++q) {
-      const uint4 v = __ldg(cs + q);
-      word[4 * q + 0] = v.x;
-      word[4 * q + 1] = v.y;
-      word[4 * q + 2] = v.z;
-      word[4 * q + 3] = v.w;
-    }
-    word[S::kWords] = __ldg(d.stream + (chunk + 1) * S::kWords);
-  }
-  w.buf = (((uint64_t)word[0] << 32) | word[1]) << gap;
+  for (int j = 0; j < S::kNB; ++j)
+    if ((uint32_t)(t + j * T) < blocks) nv[j] = __ldg(nib + t + j * T);
+
+  // K2: walk the chunk once.  Full-window lookups while every code the entry
+  // holds is sure to start before `end`, then one code at a time.
+  const uint64_t bit0 = ((uint64_t)local * T + t) * (8ull * C);
+  const uint64_t code_bits = dt->code_bits;
+  const uint64_t left = bit0 < code_bits ? code_bits - bit0 : 0;
+  const uint32_t gap = (in.gapw >> ((t & 7) * 4)) & 15u;
+  Walker w;
+  w.end = left < 8ull * C ? (int)left : 8 * C;
+  w.buf = (((uint64_t)in.w[0] << 32) | in.w[1]) << gap;
   w.valid = 64 - (int)gap;
   w.pos = (int)gap;
   w.acc = 0;
   w.nacc = 0;
   w.nw = 0;
   w.bad = false;
-  __syncthreads();  // tables ready
-
-  // K2: walk the chunk once.  Full-window lookups while every code the entry
-  // holds is sure to start before `end`, then one code at a time.
 #pragma unroll
   for (int k = 2; k <= S::kWords; ++k) {
     while (w.valid > 32 && w.pos + kK <= w.end) step_multi<C, T>(w, lut, canon, priv);
     if (w.valid > 32) break;  // at the tail with >= 20 bits buffered past `end`
-    w.buf |= (uint64_t)word[k] << (32 - w.valid);
+    w.buf |= (uint64_t)in.w[k] << (32 - w.valid);
     w.valid += 32;
   }
   while (w.pos + kK <= w.end) step_multi<C, T>(w, lut, canon, priv);
@@ -272,7 +324,6 @@ __device__ __forceinline__ void decode_group(const DevTensor& d, uint32_t g, uin
   const uint32_t total = scan[64];
   const uint32_t start = incl - cnt + scan[32 + warp];
 
-  const bool offsets_ok = off0 <= off1 && off1 <= d.n && off1 - off0 <= (uint64_t)S::kMaxCodes;
   if (any_bad || !offsets_ok || (uint64_t)total != off1 - off0) {
     if (t == 0 && status) {
       int32_t f = 0;
@@ -285,7 +336,7 @@ __device__ __forceinline__ void decode_group(const DevTensor& d, uint32_t g, uin
   }
 
   // K4a: funnel-shift this thread's exponents to stage[] nibble position
-  // (off0 mod 32) + start, so that stage word 4b.. covers output block b
+  // (off0 mod 32) + start, so that stage words 4b..4b+3 cover output block b
   const uint32_t q = (uint32_t)(off0 & 31) + start;
   const uint32_t d0 = q >> 3, dl = cnt ? (q + cnt - 1) >> 3 : 0;
   if (cnt) {
@@ -309,39 +360,16 @@ __device__ __forceinline__ void decode_group(const DevTensor& d, uint32_t g, uin
   }
   __syncthreads();
 
-  // K4b + K5: assemble 32 weights per step and store them
+  // K4b + K5
   const uint64_t base = off0 & ~31ull;
-  const uint32_t blocks = ((uint32_t)(off0 & 31) + total + 31) >> 5;
-  const uint4* nib = reinterpret_cast<const uint4*>(d.nibbles);
-  for (uint32_t b = t; b < blocks; b += T) {
-    const uint4 ex = reinterpret_cast<const uint4*>(stage)[b];
-    const uint64_t gpos = base + 32ull * b;
-    const uint4 nb = __ldg(nib + (gpos >> 5));
-    uint32_t o[8];
-    assemble8(ex.x, nb.x, o[0], o[1]);
-    assemble8(ex.y, nb.y, o[2], o[3]);
-    assemble8(ex.z, nb.z, o[4], o[5]);
-    assemble8(ex.w, nb.w, o[6], o[7]);
-    const uint64_t lo = gpos > off0 ? gpos : off0;
-    const uint64_t hi = gpos + 32 < off1 ? gpos + 32 : off1;
-    uint8_t* dst = d.out + gpos;
-    if (lo == gpos && hi == gpos + 32) {
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
-    } else {
+  const uint4* st = reinterpret_cast<const uint4*>(stage);
+  uint8_t* out = dt->out;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const uint64_t i = gpos + k;
-        if (i >= lo && i < hi) dst[k] = (uint8_t)(o[k >> 2] >> (8 * (k & 3)));
-      }
-    }
+  for (int j = 0; j < S::kNB; ++j) {
+    const uint32_t b = t + j * T;
+    if (b < blocks) store_block(out, base + 32ull * b, off0, off1, st[b], nv[j]);
   }
-}
-
-template <int C, int T>
-__global__ void __launch_bounds__(T) decode_one_kernel(const DevTensor d, int32_t* status) {
-  extern __shared__ __align__(16) uint32_t smem[];
-  decode_group<C, T>(d, blockIdx.x, smem, status);
+  for (uint32_t b = t + S::kNB * T; b < blocks; b += T) store_block(out, base + 32ull * b, off0, off1, st[b], __ldg(nib + b));
 }
 
 // the tensor whose groups contain group g: the last with group_base <= g
@@ -355,46 +383,90 @@ __device__ __forceinline__ int find_tensor(const DevTensor* ts, int count, uint3
   return lo;
 }
 
+// Persistent CTA: a contiguous run of groups (across tensors, in table order).
+// The next group's stream slice and offsets are fetched while this one is
+// decoded; the decode table is reloaded only when the run enters a new tensor.
 template <int C, int T>
-__global__ void __launch_bounds__(T) decode_many_kernel(const DevTensor* __restrict__ ts, int count, int32_t* status) {
+__device__ __forceinline__ void decode_run(const DevTensor* table, int count, uint32_t total, int32_t* status) {
+  using S = Shape<C, T>;
   extern __shared__ __align__(16) uint32_t smem[];
-  const DevTensor d = ts[find_tensor(ts, count, blockIdx.x)];
-  decode_group<C, T>(d, blockIdx.x - d.group_base, smem, status);
+  const uint32_t gb = (uint32_t)((uint64_t)blockIdx.x * total / gridDim.x);
+  const uint32_t ge = (uint32_t)((uint64_t)(blockIdx.x + 1) * total / gridDim.x);
+  if (gb >= ge) return;
+  int ti = find_tensor(table, count, gb);
+  load_tables<C, T>(table + ti, smem + S::kLutOff, reinterpret_cast<Canon*>(smem + S::kCanonOff));
+  GroupIn<C> in;
+  fetch_group<C, T>(table + ti, gb - table[ti].group_base, in);
+  for (uint32_t g = gb; g < ge; ++g) {
+    const DevTensor* dt = table + ti;
+    const uint32_t base = dt->group_base;
+    const bool more = g + 1 < ge;
+    const bool next_tensor = more && g + 1 >= base + dt->n_groups;
+    GroupIn<C> nx;
+    if (more) fetch_group<C, T>(dt + (next_tensor ? 1 : 0), g + 1 - (next_tensor ? dt[1].group_base : base), nx);
+    process_group<C, T>(dt, g - base, in, smem, status);
+    if (more) {
+      if (next_tensor) {  // every thread is past the walk of group g
+        ++ti;
+        load_tables<C, T>(table + ti, smem + S::kLutOff, reinterpret_cast<Canon*>(smem + S::kCanonOff));
+      }
+      in = nx;
+    }
+  }
+}
+
+template <int C, int T>
+__global__ void __launch_bounds__(T, Shape<C, T>::kMinBlocks) decode_table_kernel(const DevTensor* __restrict__ ts,
+                                                                                    int count, uint32_t total,
+                                                                                    int32_t* status) {
+  decode_run<C, T>(ts, count, total, status);
 }
 
 // Small batches travel inside the launch's parameter block.
-constexpr int kInlineMax = ECF8_BATCH_INLINE_MAX;
+template <int N>
 struct InlineBatch {
-  DevTensor t[kInlineMax];
+  DevTensor t[N];
   int count;
 };
+constexpr int kInlineMax = ECF8_BATCH_INLINE_MAX;
 
-template <int C, int T>
-__global__ void __launch_bounds__(T) decode_inline_kernel(const __grid_constant__ InlineBatch b, int32_t* status) {
-  extern __shared__ __align__(16) uint32_t smem[];
-  const DevTensor d = b.t[find_tensor(b.t, b.count, blockIdx.x)];
-  decode_group<C, T>(d, blockIdx.x - d.group_base, smem, status);
+template <int C, int T, int N>
+__global__ void __launch_bounds__(T, Shape<C, T>::kMinBlocks) decode_inline_kernel(
+    const __grid_constant__ InlineBatch<N> b, uint32_t total, int32_t* status) {
+  decode_run<C, T>(b.t, b.count, total, status);
 }
 
 std::atomic<uint64_t> g_launches{0};
 
+// Per device, once: allow the kernels their shared memory and size the
+// persistent grid (resident CTAs per SM x SMs).
 template <int C, int T>
-int set_smem_attr() {
-  // per device, once
-  static std::atomic<uint64_t> done_mask{0};
+int grid_for_device(uint32_t* ctas) {
+  struct Entry {
+    std::atomic<uint32_t> ctas{0};
+  };
+  static Entry per_dev[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return ECF8_ERR_CUDA;
-  const uint64_t bit = 1ull << (dev & 63);
-  if (done_mask.load() & bit) return ECF8_OK;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ECF8_ERR_CUDA;
+  uint32_t have = per_dev[dev].ctas.load();
+  if (have) {
+    *ctas = have;
+    return ECF8_OK;
+  }
   using S = Shape<C, T>;
-  if (cudaFuncSetAttribute(decode_one_kernel<C, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)S::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(decode_many_kernel<C, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)S::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(decode_inline_kernel<C, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)S::kSmemBytes) != cudaSuccess)
+  const int bytes = (int)S::kSmemBytes;
+  if (cudaFuncSetAttribute(decode_table_kernel<C, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
+      cudaFuncSetAttribute(decode_inline_kernel<C, T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
+      cudaFuncSetAttribute(decode_inline_kernel<C, T, kInlineMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bytes))
     return ECF8_ERR_CUDA;
-  done_mask.fetch_or(bit);
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_inline_kernel<C, T, kInlineMax>, T, bytes))
+    return ECF8_ERR_CUDA;
+  have = (uint32_t)(sms * (per_sm > 0 ? per_sm : 1));
+  per_dev[dev].ctas.store(have);
+  *ctas = have;
   return ECF8_OK;
 }
 
@@ -439,6 +511,25 @@ DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
 
 constexpr int kC = 32, kT = 128;  // the layout the kernels are built for
 
+// Checks one tensor of a call and appends its descriptor (skipping n = 0).
+int add_tensor(const ecf8_info* info, const void* d_blob, uint8_t* d_out, std::vector<DevTensor>& v,
+               uint64_t& groups) {
+  int rc = check_info(info);
+  if (rc) return rc;
+  if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
+  if (info->n == 0) return ECF8_OK;
+  if (!d_blob || !d_out) return ECF8_ERR_ARG;
+  if (!aligned16(d_blob) || !aligned16(d_out)) return ECF8_ERR_ALIGN;
+  DevTensor t = make_dev(info, d_blob, d_out);
+  t.group_base = (uint32_t)groups;
+  groups += info->n_groups;
+  if (groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
+  v.push_back(t);
+  return ECF8_OK;
+}
+
+uint32_t grid_size(uint32_t ctas, uint64_t groups) { return (uint32_t)(groups < ctas ? groups : ctas); }
+
 }  // namespace
 }  // namespace ecf8
 
@@ -452,16 +543,19 @@ int ecf8_layout_supported(uint32_t chunk_bytes, uint32_t group_chunks) {
 
 int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_t n, int32_t* d_status,
                 cudaStream_t s) {
-  int rc = check_info(info);
-  if (rc) return rc;
+  if (!info) return ECF8_ERR_ARG;
   if (n != info->n) return ECF8_ERR_ARG;
-  if (n == 0) return ECF8_OK;
-  if (!d_blob || !d_out) return ECF8_ERR_ARG;
-  if (!aligned16(d_blob) || !aligned16(d_out)) return ECF8_ERR_ALIGN;
-  if (!ecf8_layout_supported(info->chunk_bytes, info->group_chunks)) return ECF8_ERR_UNSUPPORTED;
-  if ((rc = set_smem_attr<kC, kT>())) return rc;
-  const DevTensor t = make_dev(info, d_blob, d_out);
-  decode_one_kernel<kC, kT><<<info->n_groups, kT, Shape<kC, kT>::kSmemBytes, s>>>(t, d_status);
+  std::vector<DevTensor> v;
+  uint64_t groups = 0;
+  int rc = add_tensor(info, d_blob, d_out, v, groups);
+  if (rc || v.empty()) return rc;
+  uint32_t ctas = 0;
+  if ((rc = grid_for_device<kC, kT>(&ctas))) return rc;
+  InlineBatch<1> b;
+  b.t[0] = v[0];
+  b.count = 1;
+  decode_inline_kernel<kC, kT, 1><<<grid_size(ctas, groups), kT, Shape<kC, kT>::kSmemBytes, s>>>(
+      b, (uint32_t)groups, d_status);
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
   return ECF8_OK;
@@ -479,37 +573,30 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
     if (!d_workspace || workspace_bytes < ecf8_batched_workspace_size(count)) return ECF8_ERR_WORKSPACE;
     if (!aligned16(d_workspace)) return ECF8_ERR_ALIGN;
   }
-  std::vector<DevTensor> host;
-  host.reserve(count);
+  std::vector<DevTensor> v;
+  v.reserve(count);
   uint64_t groups = 0;
   for (int i = 0; i < count; ++i) {
-    const ecf8_tensor& x = tensors[i];
-    int rc = check_info(x.info);
+    int rc = add_tensor(tensors[i].info, tensors[i].d_blob, tensors[i].d_out, v, groups);
     if (rc) return rc;
-    if (!ecf8_layout_supported(x.info->chunk_bytes, x.info->group_chunks)) return ECF8_ERR_UNSUPPORTED;
-    if (x.info->n == 0) continue;
-    if (!x.d_blob || !x.d_out) return ECF8_ERR_ARG;
-    if (!aligned16(x.d_blob) || !aligned16(x.d_out)) return ECF8_ERR_ALIGN;
-    DevTensor t = make_dev(x.info, x.d_blob, x.d_out);
-    t.group_base = (uint32_t)groups;
-    groups += x.info->n_groups;
-    if (groups > 0x7FFFFFFFull) return ECF8_ERR_UNSUPPORTED;
-    host.push_back(t);
   }
-  if (host.empty()) return ECF8_OK;
-  int rc = set_smem_attr<kC, kT>();
+  if (v.empty()) return ECF8_OK;
+  uint32_t ctas = 0;
+  int rc = grid_for_device<kC, kT>(&ctas);
   if (rc) return rc;
-  if (host.size() <= (size_t)kInlineMax) {
-    InlineBatch b;
-    for (size_t i = 0; i < host.size(); ++i) b.t[i] = host[i];
-    b.count = (int)host.size();
-    decode_inline_kernel<kC, kT><<<(unsigned)groups, kT, Shape<kC, kT>::kSmemBytes, s>>>(b, d_status);
+  const uint32_t grid = grid_size(ctas, groups);
+  if (v.size() <= (size_t)kInlineMax) {
+    InlineBatch<kInlineMax> b;
+    for (size_t i = 0; i < v.size(); ++i) b.t[i] = v[i];
+    b.count = (int)v.size();
+    decode_inline_kernel<kC, kT, kInlineMax><<<grid, kT, Shape<kC, kT>::kSmemBytes, s>>>(b, (uint32_t)groups,
+                                                                                          d_status);
   } else {
-    if (cudaMemcpyAsync(d_workspace, host.data(), sizeof(DevTensor) * host.size(), cudaMemcpyHostToDevice, s) !=
+    if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * v.size(), cudaMemcpyHostToDevice, s) !=
         cudaSuccess)
       return ECF8_ERR_CUDA;
-    decode_many_kernel<kC, kT><<<(unsigned)groups, kT, Shape<kC, kT>::kSmemBytes, s>>>(
-        static_cast<const DevTensor*>(d_workspace), (int)host.size(), d_status);
+    decode_table_kernel<kC, kT><<<grid, kT, Shape<kC, kT>::kSmemBytes, s>>>(
+        static_cast<const DevTensor*>(d_workspace), (int)v.size(), (uint32_t)groups, d_status);
   }
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
