@@ -72,6 +72,7 @@ extern "C" {
 #define ECF8_ERR_UNSUPPORTED (-6) /* layout the GPU kernels do not implement */
 #define ECF8_ERR_CUDA (-7)        /* a CUDA runtime call failed */
 #define ECF8_ERR_WORKSPACE (-8)   /* workspace null or too small */
+#define ECF8_ERR_TOO_MANY (-9)    /* more tensors than ecf8_decode_batched_noalloc holds */
 
 /* bits OR-ed into *d_status by the decode kernels */
 #define ECF8_STATUS_COUNT_MISMATCH 1 /* codes decoded in a group != its offset delta */
@@ -159,6 +160,33 @@ size_t ecf8_batched_workspace_size(int count);
  * the workspace must not be touched by other streams until the decode ends. */
 int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
                         int32_t* d_status, cudaStream_t s);
+
+/* Most tensors one ecf8_decode_batched_noalloc call takes. */
+#define ECF8_NOALLOC_MAX_TENSORS 1024
+
+/* ecf8_decode_batched without a workspace, for callers that cannot allocate
+ * device memory when they decode: for example a plugin running inside an
+ * inference engine that owns every device allocation and hands out no
+ * scratch, or a serving loop that must not call cudaMalloc because it
+ * synchronises the device and can stall other streams.  The paper has no
+ * counterpart of this call; it is a property of this library.
+ *
+ * The descriptor table that ecf8_decode_batched copies into the caller's
+ * workspace goes instead into one table in device memory that the library
+ * itself holds: ECF8_NOALLOC_MAX_TENSORS entries of 96 bytes (96 KB) on every
+ * GPU that loads the library, kept until the process exits.  The caller
+ * still provides every blob and output buffer.  The call makes no cudaMalloc,
+ * cudaFree or other allocating call.
+ *  - The first call on a device resolves that table's device address (and
+ *    sets the kernel attributes); make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the one table and overwrites it.  Calls
+ *    ordered on one stream are fine; calls that can overlap on the GPU
+ *    (different streams without ordering between them) race and may decode
+ *    with each other's descriptors.
+ *  - count > ECF8_NOALLOC_MAX_TENSORS returns ECF8_ERR_TOO_MANY and enqueues
+ *    nothing.  Other arguments and errors are as for ecf8_decode_batched. */
+int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count, int32_t* d_status, cudaStream_t s);
 
 /* Number of decode kernels this library has launched in this process. */
 uint64_t ecf8_launch_count(void);

@@ -18,20 +18,34 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "libecf8.so")
 
-if not os.path.exists(_SO):
-    raise ImportError(
-        f"{_SO} is missing: build it with `python -m lossless_fp8_weight_b200._build` "
-        "(or __graft_entry__.build()); the decoder has no CPU fallback")
 
+
+def _ensure_built() -> None:
+    """Compile libecf8.so in place when it is missing or older than its
+    sources (the build script is loaded by path, so this package's own import
+    does not recurse)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_ecf8_build", os.path.join(_HERE, "_build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    if mod.stale():
+        try:
+            mod.build()
+        except Exception as e:  # no toolchain: the decoder has no CPU fallback
+            raise ImportError(f"{_SO} is missing or stale and could not be built: {e}") from e
+
+
+_ensure_built()
 _lib = ctypes.CDLL(_SO)
 
 OK = 0
 ERRORS = {-1: "ARG", -2: "FORMAT", -3: "CAPACITY", -4: "CODEBOOK", -5: "ALIGN", -6: "UNSUPPORTED", -7: "CUDA",
-          -8: "WORKSPACE"}
+          -8: "WORKSPACE", -9: "TOO_MANY"}
 STATUS_COUNT_MISMATCH = 1
 STATUS_BAD_CODE = 2
 STATUS_BAD_OFFSETS = 4
 BATCH_INLINE_MAX = 64
+NOALLOC_MAX_TENSORS = 1024
 DEFAULT_CHUNK_BYTES = 32
 DEFAULT_GROUP_CHUNKS = 128
 
@@ -76,6 +90,7 @@ _lib.ecf8_decode.argtypes = [ctypes.POINTER(Info), _p, _p, _sz, _p, _p]
 _lib.ecf8_batched_workspace_size.argtypes = [_i32]
 _lib.ecf8_batched_workspace_size.restype = _sz
 _lib.ecf8_decode_batched.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p]
+_lib.ecf8_decode_batched_noalloc.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _p]
 _lib.ecf8_launch_count.restype = ctypes.c_uint64
 _lib.ecf8_strerror.restype = ctypes.c_char_p
 _lib.ecf8_strerror.argtypes = [_i32]
@@ -211,3 +226,17 @@ def decode_batched(items, workspace=None, status=None, stream=None) -> None:
         workspace, int) else 0
     _check(_lib.ecf8_decode_batched(arr, len(arr), ws, ws_bytes, _ptr(status), _stream(stream)),
            "ecf8_decode_batched")
+
+
+def decode_batched_noalloc(items, status=None, stream=None) -> None:
+    """Like decode_batched, but with no workspace: the descriptor table lives
+    in device memory the library holds (ECF8_NOALLOC_MAX_TENSORS entries), for
+    callers that cannot allocate device memory while they decode.  Calls that
+    can overlap on the GPU share that table and race; order them on one
+    stream."""
+    if isinstance(items, tuple):
+        arr = items[0]
+    else:
+        arr, _keep = make_batch(items)
+    _check(_lib.ecf8_decode_batched_noalloc(arr, len(arr), _ptr(status), _stream(stream)),
+           "ecf8_decode_batched_noalloc")

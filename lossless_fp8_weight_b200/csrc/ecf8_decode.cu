@@ -29,6 +29,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 #include <vector>
 
 #include "ecf8.h"
@@ -606,3 +607,80 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
 uint64_t ecf8_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation batched decode
+//
+// The descriptor table of ecf8_decode_batched_noalloc.  It is device memory
+// the library owns (one copy per GPU that loads the library), so callers that
+// cannot allocate need not pass a workspace.  In host code the name
+// g_noalloc_table stands for the host-side shadow of the symbol, not a device
+// address: the device address is looked up with cudaGetSymbolAddress, once
+// per device, and that pointer is what the kernel receives.  Nothing in the
+// table needs to start at zero: every call writes the entries it uses.
+namespace ecf8 {
+namespace {
+
+static __device__ __align__(256) DevTensor g_noalloc_table[ECF8_NOALLOC_MAX_TENSORS];
+
+// Device address of g_noalloc_table on the current device (resolved on the
+// first call there, with that device current).
+int noalloc_table_address(DevTensor** out) {
+  static std::atomic<DevTensor*> per_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ECF8_ERR_CUDA;
+  DevTensor* p = per_dev[dev].load();
+  if (!p) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_table) != cudaSuccess || !addr) return ECF8_ERR_CUDA;
+    p = static_cast<DevTensor*>(addr);
+    per_dev[dev].store(p);
+  }
+  *out = p;
+  return ECF8_OK;
+}
+
+}  // namespace
+}  // namespace ecf8
+
+extern "C" int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count, int32_t* d_status,
+                                           cudaStream_t s) {
+  if (count < 0 || (count > 0 && !tensors)) return ECF8_ERR_ARG;
+  if (count == 0) return ECF8_OK;
+  if (count > ECF8_NOALLOC_MAX_TENSORS) return ECF8_ERR_TOO_MANY;
+  // host staging of the descriptors: a fixed array, reused under a lock; the
+  // pageable host->device copy has read it by the time cudaMemcpyAsync returns
+  static DevTensor host_table[ECF8_NOALLOC_MAX_TENSORS];
+  static std::mutex host_lock;
+  std::lock_guard<std::mutex> guard(host_lock);
+  int used = 0;
+  uint64_t groups = 0;
+  for (int i = 0; i < count; ++i) {
+    const ecf8_info* info = tensors[i].info;
+    int rc = check_info(info);
+    if (rc) return rc;
+    if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
+    if (info->n == 0) continue;
+    if (!tensors[i].d_blob || !tensors[i].d_out) return ECF8_ERR_ARG;
+    if (!aligned16(tensors[i].d_blob) || !aligned16(tensors[i].d_out)) return ECF8_ERR_ALIGN;
+    DevTensor t = make_dev(info, tensors[i].d_blob, tensors[i].d_out);
+    t.group_base = (uint32_t)groups;
+    groups += info->n_groups;
+    if (groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
+    host_table[used++] = t;
+  }
+  if (used == 0) return ECF8_OK;
+  DevTensor* table = nullptr;
+  int rc = noalloc_table_address(&table);
+  if (rc) return rc;
+  uint32_t ctas = 0;
+  if ((rc = grid_for_device<kC, kT>(&ctas))) return rc;
+  if (cudaMemcpyAsync(table, host_table, sizeof(DevTensor) * (size_t)used, cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return ECF8_ERR_CUDA;
+  decode_table_kernel<kC, kT><<<grid_size(ctas, groups), kT, Shape<kC, kT>::kSmemBytes, s>>>(table, used,
+                                                                                              (uint32_t)groups,
+                                                                                              d_status);
+  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ECF8_OK;
+}

@@ -265,6 +265,7 @@ const char* ecf8_strerror(int code) {
     case ECF8_ERR_UNSUPPORTED: return "layout not implemented by the GPU kernels";
     case ECF8_ERR_CUDA: return "CUDA runtime error";
     case ECF8_ERR_WORKSPACE: return "workspace missing or too small";
+    case ECF8_ERR_TOO_MANY: return "more tensors than the no-allocation decode table holds";
     default: return "unknown error";
   }
 }
