@@ -47,7 +47,7 @@ STATUS_BAD_OFFSETS = 4
 BATCH_INLINE_MAX = 64
 NOALLOC_MAX_TENSORS = 1024
 DEFAULT_CHUNK_BYTES = 32
-DEFAULT_GROUP_CHUNKS = 128
+DEFAULT_GROUP_CHUNKS = 32
 
 
 class Codebook(ctypes.Structure):

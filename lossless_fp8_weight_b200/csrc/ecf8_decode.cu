@@ -5,27 +5,35 @@
 // decode_kernel pipeline; arXiv 2510.02676 abstract).  The pages' kernel is
 // prior art written for H100/RTX40 parts; this one keeps its idea -- every
 // thread owns a fixed slice of the bit stream, starts at a stored gap, counts
-// its codes, and a block-wide prefix sum of the counts places its output --
-// and is otherwise laid out for B200:
+// its codes, and a prefix sum of the counts places its output -- and is
+// otherwise laid out for B200:
 //
-//  * one CTA of T threads decodes one group of T chunks (C bytes of stream
-//    each); the group's first output index comes from the stored offsets, so
-//    CTAs never wait on each other;
-//  * each thread walks its chunk ONCE with a 4096-entry table in shared
-//    memory that yields up to six codes per lookup, and parks the exponents
-//    (4 bits each) in a thread-private, bank-interleaved smem area;
-//  * a warp-shuffle scan (plus one smem step across warps) of the per-thread
-//    code counts gives every thread its output position; threads then
-//    funnel-shift their exponents into one contiguous, 32-weight-aligned
-//    staging array;
-//  * the CTA finally streams its output range in 32-weight blocks: 16 bytes
-//    of staged exponents + one 16-byte nibble load -> 32 output bytes with
-//    byte-permute and 3-input logic ops, stored as two 16-byte vectors.
+//  * a group is 32 chunks of 32 stream bytes and belongs to ONE warp: the
+//    warp's lanes decode its chunks, a warp-shuffle scan of their code counts
+//    added to the group's stored offset places every exponent, and the warp
+//    writes the group's output.  Warps never wait for each other; the only
+//    CTA-wide barriers sit where a CTA's run of groups enters a new tensor.
+//  * decoding is a finite-state machine over bytes: a 4096-entry table in
+//    shared memory, indexed by (node of the code tree, next stream byte),
+//    gives every exponent whose code ends in that byte and the node after
+//    it.  Each lane first shifts its slice so that it starts at its first
+//    code (the gap), and zeroes the bits after its last code, so all lanes run
+//    the same fully unrolled 34-byte loop.  Zeros after a code boundary decode
+//    as repeats of the all-zero code, whose number is known and subtracted.
+//  * exponents are parked 4 bits each in lane-private shared memory, then
+//    funnel-shifted into a 32-weight-aligned stage; 16 bytes of stage plus one
+//    16-byte nibble load become 32 output bytes (byte-permute + 3-input
+//    logic), stored as two 16-byte vectors.
+//  * CTAs are persistent, one per SM, each over a contiguous run of groups;
+//    every warp fetches its next group's stream slice, gaps and offsets while
+//    it decodes the current one, and issues the current group's nibble loads
+//    before its walk.
 //
 // The path is HBM-bound integer work: no tensor cores.  Corrupt input is
 // reported through a status word; no access leaves its buffer and no loop
 // runs without a bound.
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include <atomic>
@@ -38,199 +46,149 @@
 namespace ecf8 {
 namespace {
 
-constexpr int kK = (int)kLutBits;
+// Layout the kernels implement: 32-byte chunks, 32 chunks (one warp) per group.
+constexpr int kC = 32, kT = 32;
+constexpr int kWords = kC / 4;                 // stream words per chunk
+constexpr int kSpanBits = 8 * kC;              // 256
+constexpr int kBytes = (kSpanBits + 15 + 7) / 8 + 0;  // 34: a lane may own up to 256 + 15 bits
+constexpr int kPadBits = 8 * kBytes;           // 272 bits walked by every lane
+constexpr int kPrivWords = kBytes + 1;         // parked exponent words per lane (<= 272 codes)
+constexpr int kMaxCodes = kSpanBits * kT;      // codes one group can hold: 8192
+constexpr int kStageWords = kMaxCodes / 8 + 8; // + alignment slack
+constexpr int kWarps = 16;                     // warps per CTA
+constexpr int kThreads = 32 * kWarps;
+constexpr int kNB = 8;                         // nibble blocks a lane prefetches in registers
+constexpr int kStates = 16;                    // tree nodes (<= 15 for 16 values) + the error state
+constexpr int kError = kStates - 1;
 
-template <int C, int T>
-struct Shape {
-  static_assert(C % 16 == 0 && T % 32 == 0 && T <= 1024, "unsupported layout");
-  static constexpr int kWords = C / 4;          // stream words per chunk
-  static constexpr int kPrivWords = C;          // 8C codes of 4 bits at most
-  static constexpr int kMaxCodes = 8 * C * T;   // per group
-  static constexpr int kStageWords = T * C + 8; // staged exponents, +32 for alignment
-  static constexpr int kWarps = T / 32;
-  static constexpr int kNB = 8;          // nibble blocks a thread prefetches in registers
-  static constexpr int kMinBlocks = 4;   // CTAs per SM the smem budget allows
-  // shared memory carve-up, in 32-bit words
-  static constexpr int kLutOff = 0;
-  static constexpr int kPrivOff = kLutOff + (int)kLutEntries;
-  static constexpr int kStageOff = kPrivOff + kPrivWords * T;
-  static constexpr int kScanOff = kStageOff + kStageWords;
-  static constexpr int kCanonOff = kScanOff + 72;  // warp sums, exclusive prefixes, total
-  static constexpr int kCanonWords = 17 * 3 + 4 + 4;  // first, count, base; sorted[16]; len[16]
-  static constexpr size_t kSmemBytes = 4ull * (kCanonOff + kCanonWords);
-};
-
-// Canonical decoding tables for codes longer than the 12-bit window (rare).
-struct Canon {
-  uint32_t first[17];
-  uint32_t count[17];
-  uint32_t base[17];
+// Shared memory of one CTA.  Every member read as a 16-byte vector starts on
+// a 16-byte boundary (checked below).
+struct alignas(16) Tree {
+  uint32_t first[17], count[17], base[17];  // canonical code per length
+  uint32_t nint[17], ibase[17];             // internal nodes per depth, their first state id
+  uint32_t nstates, max_len, ok;
   uint8_t sorted[16];
-  uint8_t len[16];
+  uint16_t zero_codes[kPadBits + 1];         // codes in k zero bits after a code boundary
 };
+struct alignas(16) WarpArea {
+  uint32_t priv[kPrivWords * 32];  // word k of lane l at k*32 + l
+  uint32_t stage[kStageWords];     // read as uint4 per 32-weight block
+};
+struct alignas(16) Smem {
+  uint2 fsm[kStates * 256];  // x: exponents (4 bits each, first lowest); y: byte0 next state, byte1 4*count
+  Tree tree;
+  WarpArea warp[kWarps];
+};
+static_assert(offsetof(WarpArea, stage) % 16 == 0, "stage must be 16-byte aligned");
+static_assert(sizeof(WarpArea) % 16 == 0, "warp areas must stay 16-byte aligned");
+static_assert(offsetof(Smem, warp) % 16 == 0, "warp areas must be 16-byte aligned");
+static_assert(offsetof(Smem, fsm) % 16 == 0, "table must be aligned");
+static_assert(sizeof(Smem) <= 227 * 1024, "shared memory budget");
 
-__device__ __forceinline__ void build_canon(const uint8_t* len, Canon* c) {
-  uint32_t cnt[17] = {};
-  for (int s = 0; s < 16; ++s) cnt[len[s]]++;
-  cnt[0] = 0;
-  uint32_t code = 0, base = 0;
-  for (int l = 1; l <= 16; ++l) {
-    code = (code + cnt[l - 1]) << 1;
-    c->first[l] = code;
-    c->count[l] = cnt[l];
-    c->base[l] = base;
-    base += cnt[l];
+// ---------------------------------------------------------------- decode tables
+
+// Canonical code, internal-node numbering and the zero-run table (one thread).
+__device__ void build_tree(const uint8_t* len, Tree* t) {
+  uint32_t count[17] = {};
+  uint32_t max_len = 0, present = 0;
+  uint64_t kraft = 0;
+  for (int s = 0; s < 16; ++s) {
+    const uint32_t l = len[s];
+    if (l) {
+      count[l]++;
+      present++;
+      kraft += 1ull << (16 - l);
+      max_len = l > max_len ? l : max_len;
+    }
   }
-  c->first[0] = c->count[0] = c->base[0] = 0;
-  uint32_t k = 0;
-  for (int l = 1; l <= 16; ++l)
+  uint32_t code = 0, base = 0, k = 0;
+  for (int l = 1; l <= 16; ++l) {
+    code = (code + count[l - 1]) << 1;
+    t->first[l] = code;
+    t->count[l] = count[l];
+    t->base[l] = base;
+    base += count[l];
     for (int s = 0; s < 16; ++s)
-      if (len[s] == l) c->sorted[k++] = (uint8_t)s;
-  for (int s = 0; s < 16; ++s) c->len[s] = len[s];
+      if (len[s] == l) t->sorted[k++] = (uint8_t)s;
+  }
+  t->first[0] = t->count[0] = t->base[0] = 0;
+  // internal nodes: the root, then at depth l the 2*nint[l-1] - count[l]
+  // children that are not codes (a complete code has no other kind)
+  int ok = present == 1 || kraft == (1ull << 16);
+  t->nint[0] = 1;
+  t->ibase[0] = 0;
+  uint32_t states = 1;
+  for (uint32_t l = 1; l <= 16; ++l) {
+    int64_t n = l < max_len ? 2 * (int64_t)t->nint[l - 1] - count[l] : 0;
+    if (n < 0) { ok = 0; n = 0; }
+    t->nint[l] = (uint32_t)n;
+    t->ibase[l] = states;
+    states += (uint32_t)n;
+  }
+  if (states > kStates - 1) ok = 0;
+  t->nstates = states;
+  t->max_len = max_len;
+  t->ok = ok;
+  // the all-zero path from the root meets a code after lmin zeros
+  uint32_t lmin = 16;
+  for (int l = 16; l >= 1; --l)
+    if (count[l]) lmin = l;
+  for (int z = 0; z <= kPadBits; ++z) t->zero_codes[z] = (uint16_t)(z / lmin);
 }
 
-// bitselect: bits of a where m is set, bits of b elsewhere (one LOP3)
+// One table entry: start at tree node `state`, feed the 8 bits of `byte`.
+__device__ uint2 fsm_entry(const Tree* t, uint32_t state, uint32_t byte) {
+  if (!t->ok || state >= t->nstates) return make_uint2(0, kError);
+  // node (v, l) of this state
+  uint32_t l = 0, v = 0;
+  for (uint32_t d = 1; d < t->max_len; ++d)
+    if (state >= t->ibase[d] && state < t->ibase[d] + t->nint[d]) {
+      l = d;
+      v = t->first[d] + t->count[d] + (state - t->ibase[d]);
+    }
+  uint32_t syms = 0, n = 0;
+  for (int i = 7; i >= 0; --i) {
+    v = 2 * v + ((byte >> i) & 1u);
+    ++l;
+    const uint32_t r = v - t->first[l];
+    if (r < t->count[l]) {  // a code ends here
+      syms |= (uint32_t)t->sorted[t->base[l] + r] << (4 * n);
+      ++n;
+      v = 0;
+      l = 0;
+    } else if (l >= t->max_len) {
+      return make_uint2(0, kError);
+    }
+  }
+  const uint32_t next = l == 0 ? 0 : t->ibase[l] + (v - t->first[l] - t->count[l]);
+  return make_uint2(syms, next | ((4 * n) << 8));
+}
+
+// K0: the tensor's tables into shared memory (all threads of the CTA).
+__device__ void load_tables(const DevTensor* dt, Smem* sm) {
+  __syncthreads();  // every warp is done with the previous tensor's tables
+  if (threadIdx.x == 0) build_tree(dt->len, &sm->tree);
+  __syncthreads();
+  for (int e = threadIdx.x; e < kStates * 256; e += kThreads) sm->fsm[e] = fsm_entry(&sm->tree, e >> 8, e & 255);
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- assembly
+
 __device__ __forceinline__ uint32_t bsel(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
 
 // 8 weights: E = their exponents, 4 bits each in order; N = their nibble
 // word (weight k<4 in byte k low half, weight 4+k in byte k high half).
 __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, uint32_t& hi) {
+  const uint32_t ev = (E << 3) & 0x78787878u;  // e0 e2 e4 e6 at bits 3-6 of bytes 0-3
+  const uint32_t od = (E >> 1) & 0x78787878u;  // e1 e3 e5 e7
   const uint32_t n_lo = bsel(0x80808080u, N << 4, N);  // sign to bit 7, mantissa in bits 0-2
   const uint32_t n_hi = bsel(0x80808080u, N, N >> 4);
-  const uint32_t x_lo = __byte_perm(E, 0, 0x1100);     // bytes e1e0 e1e0 e3e2 e3e2
-  const uint32_t x_hi = __byte_perm(E, 0, 0x3322);
-  const uint32_t e_lo = bsel(0x00FF00FFu, x_lo << 3, x_lo >> 1);  // even bytes low nibble, odd high
-  const uint32_t e_hi = bsel(0x00FF00FFu, x_hi << 3, x_hi >> 1);
-  lo = bsel(0x78787878u, e_lo, n_lo);
-  hi = bsel(0x78787878u, e_hi, n_hi);
+  lo = __byte_perm(ev, od, 0x5140) | (n_lo & 0x87878787u);
+  hi = __byte_perm(ev, od, 0x7362) | (n_hi & 0x87878787u);
 }
 
-struct Walker {
-  uint64_t buf;  // next stream bits, MSB-aligned
-  int valid;     // bits of buf that are stream bits
-  int pos;       // chunk-relative bit of the next code start
-  int end;       // decode codes starting before this bit
-  uint64_t acc;  // exponents not yet parked, 4 bits each, first in the low bits
-  int nacc;
-  int nw;        // words parked
-  bool bad;
-};
-
-template <int C, int T>
-__device__ __forceinline__ void park(Walker& w, uint32_t* priv, uint32_t syms, int cnt) {
-  using S = Shape<C, T>;
-  w.acc |= (uint64_t)syms << (4 * w.nacc);
-  w.nacc += cnt;
-  if (w.nacc >= 8) {
-    priv[min(w.nw, S::kPrivWords - 1) * T + threadIdx.x] = (uint32_t)w.acc;
-    w.nw++;
-    w.acc >>= 32;
-    w.nacc -= 8;
-  }
-}
-
-// One code by canonical decoding of a 16-bit window; false on bits that
-// match no code (a corrupt stream, or a one-code book seeing a 1).
-__device__ __forceinline__ bool canon_one(const Canon* c, uint64_t buf, uint32_t& sym, int& len) {
-  const uint32_t win = (uint32_t)(buf >> 48);
-#pragma unroll 1
-  for (int l = 1; l <= 16; ++l) {
-    const uint32_t v = (win >> (16 - l)) - c->first[l];
-    if (v < c->count[l]) {
-      sym = c->sorted[c->base[l] + v];
-      len = l;
-      return true;
-    }
-  }
-  return false;
-}
-
-template <int C, int T>
-__device__ __forceinline__ void step_multi(Walker& w, const uint32_t* lut, const Canon* canon, uint32_t* priv) {
-  const uint32_t e = lut[(uint32_t)(w.buf >> (64 - kK))];
-  const int cnt = (e >> 4) & 7, nb = e & 15;
-  if (cnt != 0 && nb != 0) {
-    park<C, T>(w, priv, e >> 8, cnt);
-    w.buf <<= nb;
-    w.valid -= nb;
-    w.pos += nb;
-    return;
-  }
-  uint32_t sym;
-  int len;
-  if (!canon_one(canon, w.buf, sym, len)) {
-    w.bad = true;
-    w.end = w.pos;  // stop this thread
-    return;
-  }
-  park<C, T>(w, priv, sym, 1);
-  w.buf <<= len;
-  w.valid -= len;
-  w.pos += len;
-}
-
-template <int C, int T>
-__device__ __forceinline__ void step_single(Walker& w, const uint32_t* lut, const Canon* canon, uint32_t* priv) {
-  const uint32_t e = lut[(uint32_t)(w.buf >> (64 - kK))];
-  uint32_t sym = (e >> 8) & 15;
-  int len = canon->len[sym];
-  if (((e >> 4) & 7) == 0 || len == 0) {
-    if (!canon_one(canon, w.buf, sym, len)) {
-      w.bad = true;
-      w.end = w.pos;
-      return;
-    }
-  }
-  park<C, T>(w, priv, sym, 1);
-  w.buf <<= len;
-  w.valid -= len;
-  w.pos += len;
-}
-
-// ---------------------------------------------------------------- per group
-
-// What one thread fetches ahead for a group: its stream slice (+ the next
-// word, for a code that straddles the slice end), the raw gap word, and the
-// group's two offsets.  Kept raw so the loads stay in flight until used.
-template <int C>
-struct GroupIn {
-  uint32_t w[C / 4 + 1];
-  uint32_t gapw;
-  uint64_t off0, off1;
-};
-
-template <int C, int T>
-__device__ __forceinline__ void fetch_group(const DevTensor* dt, uint32_t local, GroupIn<C>& in) {
-  using S = Shape<C, T>;
-  const uint64_t chunk = (uint64_t)local * T + threadIdx.x;
-  const uint32_t* stream = dt->stream;
-  const uint4* cs = reinterpret_cast<const uint4*>(stream + chunk * S::kWords);
-#pragma unroll
-  for (int q = 0; q < S::kWords / 4; ++q) {
-    const uint4 v = __ldg(cs + q);
-    in.w[4 * q + 0] = v.x;
-    in.w[4 * q + 1] = v.y;
-    in.w[4 * q + 2] = v.z;
-    in.w[4 * q + 3] = v.w;
-  }
-  in.w[S::kWords] = __ldg(stream + (chunk + 1) * S::kWords);
-  in.gapw = __ldg(dt->gaps + (chunk >> 3));
-  in.off0 = __ldg(dt->groups + local);
-  in.off1 = __ldg(dt->groups + local + 1);
-}
-
-// K0: the tensor's decode table and canonical tables into shared memory.
-template <int C, int T>
-__device__ __forceinline__ void load_tables(const DevTensor* dt, uint32_t* lut, Canon* canon) {
-  const uint4* src = reinterpret_cast<const uint4*>(dt->lut);
-  uint4* dst = reinterpret_cast<uint4*>(lut);
-#pragma unroll 4
-  for (int i = threadIdx.x; i < (int)kLutEntries / 4; i += T) dst[i] = __ldg(src + i);
-  if (threadIdx.x == 0) build_canon(dt->len, canon);
-  __syncthreads();
-}
-
-// K4b + K5 for one 32-weight block: staged exponents + nibbles -> 32 bytes.
+// 32 weights: 16 bytes of staged exponents + 16 bytes of nibbles -> out.
 __device__ __forceinline__ void store_block(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1, const uint4 ex,
                                             const uint4 nb) {
   uint32_t o[8];
@@ -251,106 +209,144 @@ __device__ __forceinline__ void store_block(uint8_t* out, uint64_t gpos, uint64_
   }
 }
 
-template <int C, int T>
-__device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t local, const GroupIn<C>& in, uint32_t* sm,
-                                              int32_t* status) {
-  using S = Shape<C, T>;
-  uint32_t* lut = sm + S::kLutOff;
-  uint32_t* priv = sm + S::kPrivOff;
-  uint32_t* stage = sm + S::kStageOff;
-  uint32_t* scan = sm + S::kScanOff;
-  const Canon* canon = reinterpret_cast<const Canon*>(sm + S::kCanonOff);
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+// ---------------------------------------------------------------- one group per warp
+
+// What a lane fetches ahead for a group: its slice + the next word (a code
+// may run past the slice end), the raw gap word(s), the group's offsets.
+// Kept raw so the loads stay in flight until used.
+struct GroupIn {
+  uint32_t w[kWords + 1];
+  uint32_t gapw, gapn;
+  uint64_t off0, off1;
+};
+
+__device__ __forceinline__ void fetch_group(const DevTensor* dt, uint32_t local, GroupIn& in) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint64_t chunk = (uint64_t)local * kT + lane;
+  const uint32_t* stream = dt->stream;
+  const uint4* cs = reinterpret_cast<const uint4*>(stream + chunk * kWords);
+#pragma unroll
+  for (int q = 0; q < kWords / 4; ++q) {
+    const uint4 v = __ldg(cs + q);
+    in.w[4 * q + 0] = v.x;
+    in.w[4 * q + 1] = v.y;
+    in.w[4 * q + 2] = v.z;
+    in.w[4 * q + 3] = v.w;
+  }
+  in.w[kWords] = __ldg(stream + (chunk + 1) * kWords);
+  in.gapw = __ldg(dt->gaps + (chunk >> 3));
+  // the first gap of the next group (lane 31's right neighbour), if it exists
+  in.gapn = (lane == 31 && local + 1 < dt->n_groups) ? __ldg(dt->gaps + ((chunk + 1) >> 3)) : 0u;
+  in.off0 = __ldg(dt->groups + local);
+  in.off1 = __ldg(dt->groups + local + 1);
+}
+
+__device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t local, const GroupIn& in, Smem* sm,
+                                              WarpArea* wa, int32_t* status) {
+  const uint32_t lane = threadIdx.x & 31;
   const uint64_t n = dt->n;
   const uint64_t off0 = in.off0, off1 = in.off1;
-  const bool offsets_ok = off0 <= off1 && off1 <= n && off1 - off0 <= (uint64_t)S::kMaxCodes;
+  const bool offsets_ok = off0 <= off1 && off1 <= n && off1 - off0 <= (uint64_t)kMaxCodes;
 
   // this group's nibbles: issued now, consumed after the walk
   const uint32_t blocks = offsets_ok ? (uint32_t)(((off0 & 31) + (off1 - off0) + 31) >> 5) : 0;
   const uint4* nib = reinterpret_cast<const uint4*>(dt->nibbles) + (off0 >> 5);
-  uint4 nv[S::kNB];
+  uint4 nv[kNB];
 #pragma unroll
-  for (int j = 0; j < S::kNB; ++j)
-    if ((uint32_t)(t + j * T) < blocks) nv[j] = __ldg(nib + t + j * T);
+  for (int j = 0; j < kNB; ++j)
+    if (lane + 32 * j < blocks) nv[j] = __ldg(nib + lane + 32 * j);
 
-  // K2: walk the chunk once.  Full-window lookups while every code the entry
-  // holds is sure to start before `end`, then one code at a time.
-  const uint64_t bit0 = ((uint64_t)local * T + t) * (8ull * C);
+  // K1: the lane's bits run from its first code (gap) to the next lane's
+  // first code, or to the stream end: E bits once shifted to start at 0
+  const uint32_t gap = (in.gapw >> ((lane & 7) * 4)) & 15u;
+  uint32_t gap_next = __shfl_down_sync(0xFFFFFFFFu, gap, 1);
+  if (lane == 31) gap_next = in.gapn & 15u;
+  const uint64_t bit0 = ((uint64_t)local * kT + lane) * kSpanBits;
   const uint64_t code_bits = dt->code_bits;
   const uint64_t left = bit0 < code_bits ? code_bits - bit0 : 0;
-  const uint32_t gap = (in.gapw >> ((t & 7) * 4)) & 15u;
-  Walker w;
-  w.end = left < 8ull * C ? (int)left : 8 * C;
-  w.buf = (((uint64_t)in.w[0] << 32) | in.w[1]) << gap;
-  w.valid = 64 - (int)gap;
-  w.pos = (int)gap;
-  w.acc = 0;
-  w.nacc = 0;
-  w.nw = 0;
-  w.bad = false;
+  const uint32_t stop = left < (uint64_t)(kSpanBits + gap_next) ? (uint32_t)left : kSpanBits + gap_next;
+  const uint32_t E = stop > gap ? stop - gap : 0;
+  uint32_t sw[kWords + 1];
 #pragma unroll
-  for (int k = 2; k <= S::kWords; ++k) {
-    while (w.valid > 32 && w.pos + kK <= w.end) step_multi<C, T>(w, lut, canon, priv);
-    if (w.valid > 32) break;  // at the tail with >= 20 bits buffered past `end`
-    w.buf |= (uint64_t)in.w[k] << (32 - w.valid);
-    w.valid += 32;
+  for (int i = 0; i < kWords; ++i) sw[i] = __funnelshift_l(in.w[i + 1], in.w[i], gap);
+  sw[kWords] = in.w[kWords] << gap;
+  // zero every bit at or after E (bits 32i.. of sw[i]); a lane that is not at
+  // the stream end keeps E >= 241, so only its last two words need it
+  const bool any_short = __any_sync(0xFFFFFFFFu, E < 32 * (kWords - 1));
+#pragma unroll
+  for (int i = 0; i <= kWords; ++i) {
+    if (i >= kWords - 1 || any_short) {
+      const int keep = min(max((int)E - 32 * i, 0), 32);
+      sw[i] &= (uint32_t)(0xFFFFFFFF00000000ull >> keep);
+    }
   }
-  while (w.pos + kK <= w.end) step_multi<C, T>(w, lut, canon, priv);
-  while (w.pos < w.end) step_single<C, T>(w, lut, canon, priv);
-  if (w.nacc > 0) priv[min(w.nw, S::kPrivWords - 1) * T + t] = (uint32_t)w.acc;
-  const uint32_t cnt = (uint32_t)(w.nw * 8 + w.nacc);
-  const bool overflow = w.nw > S::kPrivWords || (w.nw == S::kPrivWords && w.nacc > 0);
 
-  // K3: place -- warp-shuffle inclusive scan, then across warps
+  // K2: the byte machine.  Every lane walks 272 bits; codes completed in the
+  // zero bits after E are repeats of the all-zero code and are subtracted.
+  uint32_t* priv = wa->priv + lane;
+  uint32_t y = 0;  // previous entry: byte0 = tree node (root), byte1 = 4 * codes
+  uint32_t acc = 0, sh = 0, words = 0;
+#pragma unroll
+  for (int j = 0; j < kBytes; ++j) {
+    const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x7740u | (3u - (j & 3)));
+    const uint2 e = sm->fsm[idx];
+    y = e.y;
+    acc |= e.x << sh;
+    const uint32_t carry = __funnelshift_l(e.x, 0u, sh);
+    sh += e.y >> 8;
+    if (sh >= 32) {
+      priv[32 * words] = acc;
+      ++words;
+      acc = carry;
+      sh -= 32;
+    }
+  }
+  if (sh) priv[32 * words] = acc;
+  const uint32_t emitted = 8 * words + sh / 4;
+  const uint32_t extra = sm->tree.zero_codes[kPadBits - E];
+  const bool bad = (y & 0xFF) == (uint32_t)kError || emitted < extra;
+  const uint32_t cnt = bad ? 0 : emitted - extra;
+
+  // K3: place -- warp-shuffle scan of the counts
   uint32_t incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += y;
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= (uint32_t)o) incl += v;
   }
-  if (lane == 31) scan[warp] = incl;
-  const int any_bad = __syncthreads_or(w.bad || overflow);
-  if (warp == 0) {
-    const uint32_t v = lane < S::kWarps ? scan[lane] : 0;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane < S::kWarps) scan[32 + lane] = x - v;
-    if (lane == S::kWarps - 1) scan[64] = x;
-  }
-  __syncthreads();
-  const uint32_t total = scan[64];
-  const uint32_t start = incl - cnt + scan[32 + warp];
-
+  const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  const uint32_t start = incl - cnt;
+  const bool any_bad = __any_sync(0xFFFFFFFFu, bad);
   if (any_bad || !offsets_ok || (uint64_t)total != off1 - off0) {
-    if (t == 0 && status) {
+    if (lane == 0 && status) {
       int32_t f = 0;
       if (any_bad) f |= ECF8_STATUS_BAD_CODE;
       if (!offsets_ok) f |= ECF8_STATUS_BAD_OFFSETS;
       else if ((uint64_t)total != off1 - off0) f |= ECF8_STATUS_COUNT_MISMATCH;
       atomicOr(status, f);
     }
-    return;  // uniform across the CTA
+    return;  // uniform across the warp
   }
 
-  // K4a: funnel-shift this thread's exponents to stage[] nibble position
+  // K4a: funnel-shift this lane's exponents to stage nibble position
   // (off0 mod 32) + start, so that stage words 4b..4b+3 cover output block b
+  uint32_t* stage = wa->stage;
   const uint32_t q = (uint32_t)(off0 & 31) + start;
   const uint32_t d0 = q >> 3, dl = cnt ? (q + cnt - 1) >> 3 : 0;
   if (cnt) {
     stage[d0] = 0;
     stage[dl] = 0;
   }
-  __syncthreads();
+  __syncwarp();
   if (cnt) {
     const uint32_t r = (q & 7) * 4;
     const uint32_t used = (cnt + 7) / 8;
+    // the last parked word may hold padding codes after the lane's own ones
+    const uint32_t tail_mask = (cnt & 7) ? (1u << (4 * (cnt & 7))) - 1 : 0xFFFFFFFFu;
     uint32_t prev = 0;
     for (uint32_t j = 0; j <= dl - d0; ++j) {
-      const uint32_t cur = j < used ? priv[j * T + t] : 0;
+      uint32_t cur = j < used ? priv[32 * j] : 0;
+      if (j + 1 == used) cur &= tail_mask;
       const uint32_t v = __funnelshift_l(prev, cur, r);
       prev = cur;
       if (j == 0 || j == dl - d0)
@@ -359,18 +355,19 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
         stage[d0 + j] = v;
     }
   }
-  __syncthreads();
+  __syncwarp();
 
   // K4b + K5
   const uint64_t base = off0 & ~31ull;
   const uint4* st = reinterpret_cast<const uint4*>(stage);
   uint8_t* out = dt->out;
 #pragma unroll
-  for (int j = 0; j < S::kNB; ++j) {
-    const uint32_t b = t + j * T;
+  for (int j = 0; j < kNB; ++j) {
+    const uint32_t b = lane + 32 * j;
     if (b < blocks) store_block(out, base + 32ull * b, off0, off1, st[b], nv[j]);
   }
-  for (uint32_t b = t + S::kNB * T; b < blocks; b += T) store_block(out, base + 32ull * b, off0, off1, st[b], __ldg(nib + b));
+  for (uint32_t b = lane + 32 * kNB; b < blocks; b += 32) store_block(out, base + 32ull * b, off0, off1, st[b], __ldg(nib + b));
+  __syncwarp();  // the stage and private words are reused by this warp's next group
 }
 
 // the tensor whose groups contain group g: the last with group_base <= g
@@ -384,43 +381,44 @@ __device__ __forceinline__ int find_tensor(const DevTensor* ts, int count, uint3
   return lo;
 }
 
-// Persistent CTA: a contiguous run of groups (across tensors, in table order).
-// The next group's stream slice and offsets are fetched while this one is
-// decoded; the decode table is reloaded only when the run enters a new tensor.
-template <int C, int T>
+// Persistent CTA over a contiguous run of groups (across tensors, in table
+// order).  Within each tensor's part of the run, warp w takes groups w, w+W,
+// ... and fetches its next group while decoding the current one.
 __device__ __forceinline__ void decode_run(const DevTensor* table, int count, uint32_t total, int32_t* status) {
-  using S = Shape<C, T>;
-  extern __shared__ __align__(16) uint32_t smem[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Smem* sm = reinterpret_cast<Smem*>(smem_raw);
   const uint32_t gb = (uint32_t)((uint64_t)blockIdx.x * total / gridDim.x);
   const uint32_t ge = (uint32_t)((uint64_t)(blockIdx.x + 1) * total / gridDim.x);
   if (gb >= ge) return;
+  const uint32_t warp = threadIdx.x >> 5;
+  WarpArea* wa = &sm->warp[warp];
   int ti = find_tensor(table, count, gb);
-  load_tables<C, T>(table + ti, smem + S::kLutOff, reinterpret_cast<Canon*>(smem + S::kCanonOff));
-  GroupIn<C> in;
-  fetch_group<C, T>(table + ti, gb - table[ti].group_base, in);
-  for (uint32_t g = gb; g < ge; ++g) {
+  uint32_t g0 = gb;
+  while (g0 < ge) {
     const DevTensor* dt = table + ti;
-    const uint32_t base = dt->group_base;
-    const bool more = g + 1 < ge;
-    const bool next_tensor = more && g + 1 >= base + dt->n_groups;
-    GroupIn<C> nx;
-    if (more) fetch_group<C, T>(dt + (next_tensor ? 1 : 0), g + 1 - (next_tensor ? dt[1].group_base : base), nx);
-    process_group<C, T>(dt, g - base, in, smem, status);
-    if (more) {
-      if (next_tensor) {  // every thread is past the walk of group g
-        ++ti;
-        load_tables<C, T>(table + ti, smem + S::kLutOff, reinterpret_cast<Canon*>(smem + S::kCanonOff));
+    const uint32_t tb = dt->group_base, te = tb + dt->n_groups;
+    const uint32_t g1 = te < ge ? te : ge;  // this tensor's part of the run: [g0, g1)
+    load_tables(dt, sm);
+    uint32_t g = g0 + warp;
+    if (g < g1) {
+      GroupIn in;
+      fetch_group(dt, g - tb, in);
+      for (; g < g1; g += kWarps) {
+        GroupIn nx;
+        const bool more = g + kWarps < g1;
+        if (more) fetch_group(dt, g + kWarps - tb, nx);
+        process_group(dt, g - tb, in, sm, wa, status);
+        if (more) in = nx;
       }
-      in = nx;
     }
+    g0 = g1;
+    ++ti;
   }
 }
 
-template <int C, int T>
-__global__ void __launch_bounds__(T, Shape<C, T>::kMinBlocks) decode_table_kernel(const DevTensor* __restrict__ ts,
-                                                                                    int count, uint32_t total,
-                                                                                    int32_t* status) {
-  decode_run<C, T>(ts, count, total, status);
+__global__ void __launch_bounds__(kThreads, 1) decode_table_kernel(const DevTensor* __restrict__ ts, int count,
+                                                                    uint32_t total, int32_t* status) {
+  decode_run(ts, count, total, status);
 }
 
 // Small batches travel inside the launch's parameter block.
@@ -431,17 +429,14 @@ struct InlineBatch {
 };
 constexpr int kInlineMax = ECF8_BATCH_INLINE_MAX;
 
-template <int C, int T, int N>
-__global__ void __launch_bounds__(T, Shape<C, T>::kMinBlocks) decode_inline_kernel(
-    const __grid_constant__ InlineBatch<N> b, uint32_t total, int32_t* status) {
-  decode_run<C, T>(b.t, b.count, total, status);
+template <int N>
+__global__ void __launch_bounds__(kThreads, 1) decode_inline_kernel(const __grid_constant__ InlineBatch<N> b,
+                                                                     uint32_t total, int32_t* status) {
+  decode_run(b.t, b.count, total, status);
 }
 
 std::atomic<uint64_t> g_launches{0};
 
-// Per device, once: allow the kernels their shared memory and size the
-// persistent grid (resident CTAs per SM x SMs).
-template <int C, int T>
 int grid_for_device(uint32_t* ctas) {
   struct Entry {
     std::atomic<uint32_t> ctas{0};
@@ -454,16 +449,14 @@ int grid_for_device(uint32_t* ctas) {
     *ctas = have;
     return ECF8_OK;
   }
-  using S = Shape<C, T>;
-  const int bytes = (int)S::kSmemBytes;
-  if (cudaFuncSetAttribute(decode_table_kernel<C, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
-      cudaFuncSetAttribute(decode_inline_kernel<C, T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
-      cudaFuncSetAttribute(decode_inline_kernel<C, T, kInlineMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           bytes))
+  const int bytes = (int)sizeof(Smem);
+  if (cudaFuncSetAttribute(decode_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
+      cudaFuncSetAttribute(decode_inline_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
+      cudaFuncSetAttribute(decode_inline_kernel<kInlineMax>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))
     return ECF8_ERR_CUDA;
   int sms = 0, per_sm = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_inline_kernel<C, T, kInlineMax>, T, bytes))
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_inline_kernel<kInlineMax>, kThreads, bytes))
     return ECF8_ERR_CUDA;
   have = (uint32_t)(sms * (per_sm > 0 ? per_sm : 1));
   per_dev[dev].ctas.store(have);
@@ -490,6 +483,11 @@ int check_info(const ecf8_info* info) {
     if (info->len[s]) kraft += 1ull << (16 - info->len[s]);
   }
   if (kraft > (1ull << 16) || (info->n && kraft == 0)) return ECF8_ERR_CODEBOOK;
+  // the decoder's state machine needs a complete code (Kraft sum 1) or a
+  // single value, which is what the encoder always writes
+  int present = 0;
+  for (int s = 0; s < 16; ++s) present += info->len[s] ? 1 : 0;
+  if (info->n && present > 1 && kraft != (1ull << 16)) return ECF8_ERR_CODEBOOK;
   return ECF8_OK;
 }
 
@@ -509,8 +507,6 @@ DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
   for (int s = 0; s < 16; ++s) t.len[s] = info->len[s];
   return t;
 }
-
-constexpr int kC = 32, kT = 128;  // the layout the kernels are built for
 
 // Checks one tensor of a call and appends its descriptor (skipping n = 0).
 int add_tensor(const ecf8_info* info, const void* d_blob, uint8_t* d_out, std::vector<DevTensor>& v,
@@ -551,11 +547,11 @@ int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_
   int rc = add_tensor(info, d_blob, d_out, v, groups);
   if (rc || v.empty()) return rc;
   uint32_t ctas = 0;
-  if ((rc = grid_for_device<kC, kT>(&ctas))) return rc;
+  if ((rc = grid_for_device(&ctas))) return rc;
   InlineBatch<1> b;
   b.t[0] = v[0];
   b.count = 1;
-  decode_inline_kernel<kC, kT, 1><<<grid_size(ctas, groups), kT, Shape<kC, kT>::kSmemBytes, s>>>(
+  decode_inline_kernel<1><<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(
       b, (uint32_t)groups, d_status);
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -583,20 +579,20 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
   }
   if (v.empty()) return ECF8_OK;
   uint32_t ctas = 0;
-  int rc = grid_for_device<kC, kT>(&ctas);
+  int rc = grid_for_device(&ctas);
   if (rc) return rc;
   const uint32_t grid = grid_size(ctas, groups);
   if (v.size() <= (size_t)kInlineMax) {
     InlineBatch<kInlineMax> b;
     for (size_t i = 0; i < v.size(); ++i) b.t[i] = v[i];
     b.count = (int)v.size();
-    decode_inline_kernel<kC, kT, kInlineMax><<<grid, kT, Shape<kC, kT>::kSmemBytes, s>>>(b, (uint32_t)groups,
+    decode_inline_kernel<kInlineMax><<<grid, kThreads, sizeof(Smem), s>>>(b, (uint32_t)groups,
                                                                                           d_status);
   } else {
     if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * v.size(), cudaMemcpyHostToDevice, s) !=
         cudaSuccess)
       return ECF8_ERR_CUDA;
-    decode_table_kernel<kC, kT><<<grid, kT, Shape<kC, kT>::kSmemBytes, s>>>(
+    decode_table_kernel<<<grid, kThreads, sizeof(Smem), s>>>(
         static_cast<const DevTensor*>(d_workspace), (int)v.size(), (uint32_t)groups, d_status);
   }
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
@@ -673,11 +669,11 @@ extern "C" int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count
   int rc = noalloc_table_address(&table);
   if (rc) return rc;
   uint32_t ctas = 0;
-  if ((rc = grid_for_device<kC, kT>(&ctas))) return rc;
+  if ((rc = grid_for_device(&ctas))) return rc;
   if (cudaMemcpyAsync(table, host_table, sizeof(DevTensor) * (size_t)used, cudaMemcpyHostToDevice, s) !=
       cudaSuccess)
     return ECF8_ERR_CUDA;
-  decode_table_kernel<kC, kT><<<grid_size(ctas, groups), kT, Shape<kC, kT>::kSmemBytes, s>>>(table, used,
+  decode_table_kernel<<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(table, used,
                                                                                               (uint32_t)groups,
                                                                                               d_status);
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;

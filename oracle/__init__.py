@@ -128,7 +128,7 @@ def lut_entry(lengths, pattern: int) -> int:
     return int(_load().oracle_lut_entry(ln.ctypes.data, pattern))
 
 
-def encode(x, lengths=None, chunk_bytes: int = 32, group_chunks: int = 128, max_len: int = 16) -> np.ndarray:
+def encode(x, lengths=None, chunk_bytes: int = 32, group_chunks: int = 32, max_len: int = 16) -> np.ndarray:
     """Blob for ``x`` (uint8 E4M3 bytes).  Lengths default to the code built
     from ``x``'s own exponent histogram."""
     x = _u8(x)

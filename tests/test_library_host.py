@@ -45,7 +45,7 @@ def test_abi_version_and_strerror(L):
 
 
 @pytest.mark.parametrize("n", [0, 1, 2, 3, 7, 31, 32, 33, 4095, 4096, 4097, 65537])
-@pytest.mark.parametrize("layout", [(32, 128), (4, 1), (16, 3), (8, 5), (64, 64)])
+@pytest.mark.parametrize("layout", [(32, 32), (32, 128), (4, 1), (16, 3), (8, 5), (64, 64)])
 def test_encoder_bytes_equal_oracle(L, n, layout):
     x = synth.single_normal_1k().tensors[0].generate(count=n) if n else np.zeros(0, np.uint8)
     C, T = layout
@@ -130,7 +130,8 @@ def test_encode_rejects_bad_codebooks(L):
 
 
 def test_layout_support_and_workspace_sizes(L):
-    assert L.layout_supported(32, 128)
+    assert L.layout_supported(32, 32)
+    assert not L.layout_supported(32, 128)
     assert not L.layout_supported(4, 1)
     assert L.batched_workspace_size(1) == 0 and L.batched_workspace_size(64) == 0
     assert L.batched_workspace_size(65) == 65 * 96

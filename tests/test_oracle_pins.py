@@ -286,7 +286,7 @@ EDGE_SIZES = [0, 1, 2, 3, 7, 8, 31, 32, 33, 4095, 4096, 4097]
 @pytest.mark.parametrize("n", EDGE_SIZES)
 def test_round_trip_edge_sizes(n):
     x = synth.single_normal_1k().tensors[0].generate(count=n) if n else np.zeros(0, np.uint8)
-    for C, T in [(32, 128), (4, 1), (16, 3)]:
+    for C, T in [(32, 32), (32, 128), (4, 1), (16, 3)]:
         blob = oracle.encode(x, chunk_bytes=C, group_chunks=T)
         assert np.array_equal(oracle.decode(blob, n), x)
         assert oracle.check_index(blob) == 0
