@@ -66,8 +66,10 @@ constexpr int kError = kStates - 1;
 struct alignas(16) Tree {
   uint32_t first[17], count[17], base[17];  // canonical code per length
   uint32_t nint[17], ibase[17];             // internal nodes per depth, their first state id
-  uint32_t nstates, max_len, ok;
+  uint32_t nstates, max_len, ok, lmin;
   uint8_t sorted[16];
+  uint16_t bit_step[kStates * 2];            // (state, bit) -> next state | symbol << 4 | emitted << 8
+  uint32_t nib_step[kStates * 16];           // (state, 4 bits) -> symbols | count << 16 | next << 20
   uint16_t zero_codes[kPadBits + 1];         // codes in k zero bits after a code boundary
 };
 struct alignas(16) WarpArea {
@@ -87,7 +89,9 @@ static_assert(sizeof(Smem) <= 227 * 1024, "shared memory budget");
 
 // ---------------------------------------------------------------- decode tables
 
-// Canonical code, internal-node numbering and the zero-run table (one thread).
+// Canonical code and internal-node numbering (one thread; a few hundred
+// instructions).  State 0 is the root; the internal nodes at depth l are the
+// values first[l] + count[l] + k, k < nint[l], numbered from ibase[l].
 __device__ void build_tree(const uint8_t* len, Tree* t) {
   uint32_t count[17] = {};
   uint32_t max_len = 0, present = 0;
@@ -101,19 +105,18 @@ __device__ void build_tree(const uint8_t* len, Tree* t) {
       max_len = l > max_len ? l : max_len;
     }
   }
-  uint32_t code = 0, base = 0, k = 0;
+  uint32_t code = 0, base = 0, k = 0, lmin = 0;
   for (int l = 1; l <= 16; ++l) {
     code = (code + count[l - 1]) << 1;
     t->first[l] = code;
     t->count[l] = count[l];
     t->base[l] = base;
     base += count[l];
+    if (count[l] && !lmin) lmin = l;
     for (int s = 0; s < 16; ++s)
       if (len[s] == l) t->sorted[k++] = (uint8_t)s;
   }
   t->first[0] = t->count[0] = t->base[0] = 0;
-  // internal nodes: the root, then at depth l the 2*nint[l-1] - count[l]
-  // children that are not codes (a complete code has no other kind)
   int ok = present == 1 || kraft == (1ull << 16);
   t->nint[0] = 1;
   t->ibase[0] = 0;
@@ -129,47 +132,56 @@ __device__ void build_tree(const uint8_t* len, Tree* t) {
   t->nstates = states;
   t->max_len = max_len;
   t->ok = ok;
-  // the all-zero path from the root meets a code after lmin zeros
-  uint32_t lmin = 16;
-  for (int l = 16; l >= 1; --l)
-    if (count[l]) lmin = l;
-  for (int z = 0; z <= kPadBits; ++z) t->zero_codes[z] = (uint16_t)(z / lmin);
+  t->lmin = lmin ? lmin : 1;  // the all-zero path from the root meets a code after lmin zeros
 }
 
-// One table entry: start at tree node `state`, feed the 8 bits of `byte`.
-__device__ uint2 fsm_entry(const Tree* t, uint32_t state, uint32_t byte) {
-  if (!t->ok || state >= t->nstates) return make_uint2(0, kError);
-  // node (v, l) of this state
+// One bit from tree node `state`: the next node, and the value whose code
+// it completes (if any); the error state absorbs everything.
+__device__ uint32_t bit_entry(const Tree* t, uint32_t state, uint32_t bit) {
+  if (!t->ok || state >= t->nstates) return kError;
   uint32_t l = 0, v = 0;
   for (uint32_t d = 1; d < t->max_len; ++d)
     if (state >= t->ibase[d] && state < t->ibase[d] + t->nint[d]) {
       l = d;
       v = t->first[d] + t->count[d] + (state - t->ibase[d]);
     }
-  uint32_t syms = 0, n = 0;
-  for (int i = 7; i >= 0; --i) {
-    v = 2 * v + ((byte >> i) & 1u);
-    ++l;
-    const uint32_t r = v - t->first[l];
-    if (r < t->count[l]) {  // a code ends here
-      syms |= (uint32_t)t->sorted[t->base[l] + r] << (4 * n);
-      ++n;
-      v = 0;
-      l = 0;
-    } else if (l >= t->max_len) {
-      return make_uint2(0, kError);
-    }
-  }
-  const uint32_t next = l == 0 ? 0 : t->ibase[l] + (v - t->first[l] - t->count[l]);
-  return make_uint2(syms, next | ((4 * n) << 8));
+  v = 2 * v + bit;
+  ++l;
+  const uint32_t r = v - t->first[l];
+  if (r < t->count[l]) return 0u | ((uint32_t)t->sorted[t->base[l] + r] << 4) | (1u << 8);  // back to the root
+  if (l >= t->max_len) return kError;
+  return t->ibase[l] + (v - t->first[l] - t->count[l]);
 }
 
-// K0: the tensor's tables into shared memory (all threads of the CTA).
+// K0: the tensor's tables into shared memory (all threads of the CTA):
+// bit steps -> 4-bit steps -> the byte table, each built from the last.
 __device__ void load_tables(const DevTensor* dt, Smem* sm) {
+  Tree* t = &sm->tree;
+  const int tid = threadIdx.x;
   __syncthreads();  // every warp is done with the previous tensor's tables
-  if (threadIdx.x == 0) build_tree(dt->len, &sm->tree);
+  if (tid == 0) build_tree(dt->len, t);
   __syncthreads();
-  for (int e = threadIdx.x; e < kStates * 256; e += kThreads) sm->fsm[e] = fsm_entry(&sm->tree, e >> 8, e & 255);
+  if (tid < kStates * 2) t->bit_step[tid] = (uint16_t)bit_entry(t, tid >> 1, tid & 1);
+  for (int z = tid; z <= kPadBits; z += kThreads) t->zero_codes[z] = (uint16_t)(z / t->lmin);
+  __syncthreads();
+  if (tid < kStates * 16) {
+    uint32_t st = tid >> 4, syms = 0, n = 0;
+    for (int i = 3; i >= 0; --i) {
+      const uint32_t e = t->bit_step[2 * st + ((tid >> i) & 1)];
+      if (e & 0x100) syms |= ((e >> 4) & 15u) << (4 * n++);
+      st = e & 15u;
+    }
+    t->nib_step[tid] = syms | (n << 16) | (st << 20);
+  }
+  __syncthreads();
+  for (int e = tid; e < kStates * 256; e += kThreads) {
+    const uint32_t a = t->nib_step[((e >> 8) << 4) | ((e >> 4) & 15)];
+    const uint32_t na = (a >> 16) & 15u, sa = a >> 20;
+    const uint32_t b = t->nib_step[(sa << 4) | (e & 15)];
+    const uint32_t nb = (b >> 16) & 15u, sb = b >> 20;
+    const uint32_t syms = (a & 0xFFFFu) | ((b & 0xFFFFu) << (4 * na));
+    sm->fsm[e] = sb == (uint32_t)kError ? make_uint2(0, kError) : make_uint2(syms, sb | ((4 * (na + nb)) << 8));
+  }
   __syncthreads();
 }
 
@@ -188,25 +200,31 @@ __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, 
   hi = __byte_perm(ev, od, 0x7362) | (n_hi & 0x87878787u);
 }
 
-// 32 weights: 16 bytes of staged exponents + 16 bytes of nibbles -> out.
-__device__ __forceinline__ void store_block(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1, const uint4 ex,
-                                            const uint4 nb) {
+// 32 weights: 16 bytes of staged exponents + 16 bytes of nibbles -> out,
+// for a block that lies wholly inside the group.
+__device__ __forceinline__ void store_block(uint8_t* out, uint64_t gpos, const uint4 ex, const uint4 nb) {
   uint32_t o[8];
   assemble8(ex.x, nb.x, o[0], o[1]);
   assemble8(ex.y, nb.y, o[2], o[3]);
   assemble8(ex.z, nb.z, o[4], o[5]);
   assemble8(ex.w, nb.w, o[6], o[7]);
-  uint8_t* dst = out + gpos;
-  if (gpos >= off0 && gpos + 32 <= off1) {
-    reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
-  } else {  // the group's ragged ends: bytes inside [off0, off1) only
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const uint64_t i = gpos + k;
-      if (i >= off0 && i < off1) dst[k] = (uint8_t)(o[k >> 2] >> (8 * (k & 3)));
-    }
-  }
+  uint4* dst = reinterpret_cast<uint4*>(out + gpos);
+  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// A block the group only partly owns (its first or last): the 32 lanes
+// write one byte each, those inside [off0, off1).  `nw` is the block's
+// nibble word for this lane's weight (word lane / 8 of the block).
+__device__ __forceinline__ void store_ragged(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1,
+                                             const uint32_t* stage, uint32_t b, uint32_t nw) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint64_t p = gpos + lane;
+  const uint32_t i = 32 * b + lane;  // stage nibble of this weight
+  const uint32_t e = (stage[i >> 3] >> (4 * (i & 7))) & 15u;
+  const uint32_t k = lane & 7;       // place within its 8-weight nibble word
+  const uint32_t v = (nw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
+  if (p >= off0 && p < off1) out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
 }
 
 // ---------------------------------------------------------------- one group per warp
@@ -329,7 +347,8 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   }
 
   // K4a: funnel-shift this lane's exponents to stage nibble position
-  // (off0 mod 32) + start, so that stage words 4b..4b+3 cover output block b
+  // (off0 mod 32) + start, so that stage words 4b..4b+3 cover output block b.
+  // Words shared with a neighbour lane are zeroed, then OR-ed atomically.
   uint32_t* stage = wa->stage;
   const uint32_t q = (uint32_t)(off0 & 31) + start;
   const uint32_t d0 = q >> 3, dl = cnt ? (q + cnt - 1) >> 3 : 0;
@@ -343,30 +362,58 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     const uint32_t used = (cnt + 7) / 8;
     // the last parked word may hold padding codes after the lane's own ones
     const uint32_t tail_mask = (cnt & 7) ? (1u << (4 * (cnt & 7))) - 1 : 0xFFFFFFFFu;
-    uint32_t prev = 0;
-    for (uint32_t j = 0; j <= dl - d0; ++j) {
+    const uint32_t nwd = dl - d0 + 1;  // destination words: used or used + 1
+    uint32_t prev = priv[0];
+    if (used == 1) prev &= tail_mask;
+    atomicOr(&stage[d0], prev << r);
+    uint32_t j = 1;
+#pragma unroll 4
+    for (; j + 1 < nwd; ++j) {  // interior words belong to this lane alone
+      uint32_t cur = priv[32 * j];
+      if (j + 1 == used) cur &= tail_mask;
+      stage[d0 + j] = __funnelshift_l(prev, cur, r);
+      prev = cur;
+    }
+    if (nwd > 1) {
       uint32_t cur = j < used ? priv[32 * j] : 0;
       if (j + 1 == used) cur &= tail_mask;
-      const uint32_t v = __funnelshift_l(prev, cur, r);
-      prev = cur;
-      if (j == 0 || j == dl - d0)
-        atomicOr(&stage[d0 + j], v);
-      else
-        stage[d0 + j] = v;
+      atomicOr(&stage[d0 + j], __funnelshift_l(prev, cur, r));
     }
   }
   __syncwarp();
 
-  // K4b + K5
+  // K4b + K5: whole blocks by their lane; the group's first and last block,
+  // when only partly its own, by the whole warp one byte per lane
   const uint64_t base = off0 & ~31ull;
   const uint4* st = reinterpret_cast<const uint4*>(stage);
   uint8_t* out = dt->out;
+  const uint32_t first_full = (off0 & 31) ? 1u : 0u;
+  const uint32_t end_full = (off1 & 31) ? blocks - 1 : blocks;  // blocks [first_full, end_full) are whole
 #pragma unroll
   for (int j = 0; j < kNB; ++j) {
     const uint32_t b = lane + 32 * j;
-    if (b < blocks) store_block(out, base + 32ull * b, off0, off1, st[b], nv[j]);
+    if (b >= first_full && b < end_full) store_block(out, base + 32ull * b, st[b], nv[j]);
   }
-  for (uint32_t b = lane + 32 * kNB; b < blocks; b += 32) store_block(out, base + 32ull * b, off0, off1, st[b], __ldg(nib + b));
+  for (uint32_t b = lane + 32 * kNB; b < end_full; b += 32) store_block(out, base + 32ull * b, st[b], __ldg(nib + b));
+  // ragged ends: the nibble word for lane's weight comes from the lane that
+  // prefetched the block, or from memory past the prefetch window
+  const uint32_t ragged[2] = {first_full ? 0u : 0xFFFFFFFFu, end_full < blocks ? blocks - 1 : 0xFFFFFFFFu};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t b = ragged[k];
+    if (b == 0xFFFFFFFFu || (k == 1 && b == ragged[0])) continue;  // uniform across the warp
+    const uint32_t owner = b & 31, slot = b >> 5;
+    uint4 v = nv[0];
+#pragma unroll
+    for (int jj = 1; jj < kNB; ++jj)
+      if ((uint32_t)jj == slot) v = nv[jj];
+    if (slot >= (uint32_t)kNB) v = __ldg(nib + b);  // every lane reads the same 16 bytes
+    const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, v.x, owner), w1 = __shfl_sync(0xFFFFFFFFu, v.y, owner);
+    const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, v.z, owner), w3 = __shfl_sync(0xFFFFFFFFu, v.w, owner);
+    const uint32_t sel = lane >> 3;
+    const uint32_t nw = sel == 0 ? w0 : sel == 1 ? w1 : sel == 2 ? w2 : w3;
+    store_ragged(out, base + 32ull * b, off0, off1, stage, b, nw);
+  }
   __syncwarp();  // the stage and private words are reused by this warp's next group
 }
 
