@@ -37,7 +37,7 @@ METRIC = "ECF8 decode GB/s (FP8 out) and % of HBM roofline on 1 B200; compressio
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SRC = os.path.join(ROOT, "lossless_fp8_weight_b200", "csrc", "ecf8_decode.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
 
 
 def workload_by_name(name: str) -> synth.Workload:
@@ -114,8 +114,12 @@ def recorded_traffic(workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source and this workload."""
     try:
+        rec = {}
         with open(TRAFFIC_FILE) as f:
-            rec = json.load(f)
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    rec[k.strip()] = v.strip()
         if rec.get("kernel_sha") == kernel_sha() and rec.get("workload") == workload_name:
             return float(rec["dram_bytes_per_launch"])
     except Exception:

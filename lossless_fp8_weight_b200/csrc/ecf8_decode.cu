@@ -21,9 +21,9 @@
 //    the same fully unrolled 34-byte loop.  Zeros after a code boundary decode
 //    as repeats of the all-zero code, whose number is known and subtracted.
 //  * exponents are parked 4 bits each in lane-private shared memory, then
-//    funnel-shifted into a 32-weight-aligned stage; 16 bytes of stage plus one
-//    16-byte nibble load become 32 output bytes (byte-permute + 3-input
-//    logic), stored as two 16-byte vectors.
+//    funnel-shifted into a 32-weight-aligned stage; 8 bytes of stage plus one
+//    8-byte nibble load become 16 output bytes (byte-permute + 3-input
+//    logic), and consecutive lanes store consecutive 16-byte vectors.
 //  * CTAs are persistent, one per SM, each over a contiguous run of groups;
 //    every warp fetches its next group's stream slice, gaps and offsets while
 //    it decodes the current one, and issues the current group's nibble loads
@@ -57,7 +57,7 @@ constexpr int kMaxCodes = kSpanBits * kT;      // codes one group can hold: 8192
 constexpr int kStageWords = kMaxCodes / 8 + 8; // + alignment slack
 constexpr int kWarps = 16;                     // warps per CTA
 constexpr int kThreads = 32 * kWarps;
-constexpr int kNB = 8;                         // nibble blocks a lane prefetches in registers
+constexpr int kNU = 16;                        // 16-weight nibble units a lane prefetches in registers
 constexpr int kStates = 16;                    // tree nodes (<= 15 for 16 values) + the error state
 constexpr int kError = kStates - 1;
 
@@ -200,31 +200,20 @@ __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, 
   hi = __byte_perm(ev, od, 0x7362) | (n_hi & 0x87878787u);
 }
 
-// 32 weights: 16 bytes of staged exponents + 16 bytes of nibbles -> out,
-// for a block that lies wholly inside the group.
-__device__ __forceinline__ void store_block(uint8_t* out, uint64_t gpos, const uint4 ex, const uint4 nb) {
-  uint32_t o[8];
-  assemble8(ex.x, nb.x, o[0], o[1]);
-  assemble8(ex.y, nb.y, o[2], o[3]);
-  assemble8(ex.z, nb.z, o[4], o[5]);
-  assemble8(ex.w, nb.w, o[6], o[7]);
-  uint4* dst = reinterpret_cast<uint4*>(out + gpos);
-  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
-// A block the group only partly owns (its first or last): the 32 lanes
-// write one byte each, those inside [off0, off1).  `nw` is the block's
-// nibble word for this lane's weight (word lane / 8 of the block).
-__device__ __forceinline__ void store_ragged(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1,
-                                             const uint32_t* stage, uint32_t b, uint32_t nw) {
+// A unit the group owns only in part (its first or last): lanes 0-15 write
+// one byte each, those inside [off0, off1).  `nw` is the unit's nibble word
+// holding this lane's weight (word (lane & 15) / 8), fetched at group start.
+__device__ __forceinline__ void ragged16(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1,
+                                         const uint32_t* stage, uint32_t u, uint32_t nw) {
   const uint32_t lane = threadIdx.x & 31;
   const uint64_t p = gpos + lane;
-  const uint32_t i = 32 * b + lane;  // stage nibble of this weight
-  const uint32_t e = (stage[i >> 3] >> (4 * (i & 7))) & 15u;
-  const uint32_t k = lane & 7;       // place within its 8-weight nibble word
-  const uint32_t v = (nw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
-  if (p >= off0 && p < off1) out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
+  if (lane < 16 && p >= off0 && p < off1) {
+    const uint32_t i = 16 * u + lane;
+    const uint32_t e = (stage[i >> 3] >> (4 * (i & 7))) & 15u;
+    const uint32_t k = lane & 7;
+    const uint32_t v = (nw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
+    out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
+  }
 }
 
 // ---------------------------------------------------------------- one group per warp
@@ -267,12 +256,23 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   const bool offsets_ok = off0 <= off1 && off1 <= n && off1 - off0 <= (uint64_t)kMaxCodes;
 
   // this group's nibbles: issued now, consumed after the walk
-  const uint32_t blocks = offsets_ok ? (uint32_t)(((off0 & 31) + (off1 - off0) + 31) >> 5) : 0;
-  const uint4* nib = reinterpret_cast<const uint4*>(dt->nibbles) + (off0 >> 5);
-  uint4 nv[kNB];
+  // (16-weight units: unit u = weights base + 16u.., 8 bytes of nibbles,
+  // base = off0 rounded down to 32); also the nibble words of the group's
+  // first and last unit when the group owns them only in part
+  const uint32_t units = offsets_ok ? (uint32_t)(((off0 & 31) + (off1 - off0) + 15) >> 4) : 0;
+  const uint2* nib = reinterpret_cast<const uint2*>(dt->nibbles) + (off0 >> 5) * 2;
+  uint2 nv[kNU];
 #pragma unroll
-  for (int j = 0; j < kNB; ++j)
-    if (lane + 32 * j < blocks) nv[j] = __ldg(nib + lane + 32 * j);
+  for (int j = 0; j < kNU; ++j)
+    if (lane + 32 * j < units) nv[j] = __ldg(nib + lane + 32 * j);
+  const uint32_t* nib32 = reinterpret_cast<const uint32_t*>(nib);
+  const uint32_t u0 = (uint32_t)(off0 & 31) >> 4;
+  const uint32_t first_full = u0 + ((off0 & 15) ? 1u : 0u);
+  const uint32_t end_full = (units && (off1 & 15)) ? units - 1 : units;
+  const bool hr = units && first_full != u0;  // units == 0 when the offsets are not to be trusted
+  const bool tr = end_full < units && !(hr && end_full == u0);
+  const uint32_t head_w = hr ? __ldg(nib32 + 2 * u0 + ((lane & 15) >> 3)) : 0u;
+  const uint32_t tail_w = tr ? __ldg(nib32 + 2 * end_full + ((lane & 15) >> 3)) : 0u;
 
   // K1: the lane's bits run from its first code (gap) to the next lane's
   // first code, or to the stream end: E bits once shifted to start at 0
@@ -382,38 +382,32 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   }
   __syncwarp();
 
-  // K4b + K5: whole blocks by their lane; the group's first and last block,
-  // when only partly its own, by the whole warp one byte per lane
+  // K4b + K5: whole units by their lane -- consecutive lanes store
+  // consecutive 16 bytes, 512 contiguous bytes per instruction; the ragged
+  // first and last unit one byte per lane
   const uint64_t base = off0 & ~31ull;
-  const uint4* st = reinterpret_cast<const uint4*>(stage);
+  const uint2* st = reinterpret_cast<const uint2*>(stage);
   uint8_t* out = dt->out;
-  const uint32_t first_full = (off0 & 31) ? 1u : 0u;
-  const uint32_t end_full = (off1 & 31) ? blocks - 1 : blocks;  // blocks [first_full, end_full) are whole
 #pragma unroll
-  for (int j = 0; j < kNB; ++j) {
-    const uint32_t b = lane + 32 * j;
-    if (b >= first_full && b < end_full) store_block(out, base + 32ull * b, st[b], nv[j]);
+  for (int j = 0; j < kNU; ++j) {
+    const uint32_t u = lane + 32 * j;
+    if (u >= first_full && u < end_full) {
+      uint32_t o[4];
+      const uint2 ex = st[u];
+      assemble8(ex.x, nv[j].x, o[0], o[1]);
+      assemble8(ex.y, nv[j].y, o[2], o[3]);
+      *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
-  for (uint32_t b = lane + 32 * kNB; b < end_full; b += 32) store_block(out, base + 32ull * b, st[b], __ldg(nib + b));
-  // ragged ends: the nibble word for lane's weight comes from the lane that
-  // prefetched the block, or from memory past the prefetch window
-  const uint32_t ragged[2] = {first_full ? 0u : 0xFFFFFFFFu, end_full < blocks ? blocks - 1 : 0xFFFFFFFFu};
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const uint32_t b = ragged[k];
-    if (b == 0xFFFFFFFFu || (k == 1 && b == ragged[0])) continue;  // uniform across the warp
-    const uint32_t owner = b & 31, slot = b >> 5;
-    uint4 v = nv[0];
-#pragma unroll
-    for (int jj = 1; jj < kNB; ++jj)
-      if ((uint32_t)jj == slot) v = nv[jj];
-    if (slot >= (uint32_t)kNB) v = __ldg(nib + b);  // every lane reads the same 16 bytes
-    const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, v.x, owner), w1 = __shfl_sync(0xFFFFFFFFu, v.y, owner);
-    const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, v.z, owner), w3 = __shfl_sync(0xFFFFFFFFu, v.w, owner);
-    const uint32_t sel = lane >> 3;
-    const uint32_t nw = sel == 0 ? w0 : sel == 1 ? w1 : sel == 2 ? w2 : w3;
-    store_ragged(out, base + 32ull * b, off0, off1, stage, b, nw);
+  for (uint32_t u = lane + 32 * kNU; u < end_full; u += 32) {
+    uint32_t o[4];
+    const uint2 ex = st[u], nb = __ldg(nib + u);
+    assemble8(ex.x, nb.x, o[0], o[1]);
+    assemble8(ex.y, nb.y, o[2], o[3]);
+    *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  if (hr) ragged16(out, base + 16ull * u0, off0, off1, stage, u0, head_w);
+  if (tr) ragged16(out, base + 16ull * end_full, off0, off1, stage, end_full, tail_w);
   __syncwarp();  // the stage and private words are reused by this warp's next group
 }
 
