@@ -264,6 +264,179 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t.cpu()]
 
 
+# ---------------------------------------------------------------- per-config sweep
+
+def _blake(a: np.ndarray) -> str:
+    return hashlib.blake2b(memoryview(np.ascontiguousarray(a)), digest_size=16).hexdigest()
+
+
+def _encode_specs(specs, L, keep=False):
+    """Generate and encode tensors one by one; keep a hash of each source."""
+    out = []
+    for t in specs:
+        x = t.generate()
+        hist = L.histogram(x)
+        blob = L.encode(x, codebook=L.build_codebook(hist))
+        info = L.blob_info(blob)
+        out.append({"name": t.name, "n": int(x.size), "blob": blob, "info": info, "hist": hist,
+                    "hash": _blake(x), "x": x if keep else None,
+                    "le6": float(hist[info.lengths.astype(np.int64) <= 6].sum()) / max(1, x.size)})
+    return out
+
+
+def _upload(torch, dev, blobs):
+    offs, o = [], 0
+    for b in blobs:
+        offs.append(o)
+        o += (b.size + 255) // 256 * 256
+    d = torch.empty(max(o, 256), dtype=torch.uint8, device=dev)
+    for b, off in zip(blobs, offs):
+        d[off:off + b.size].copy_(torch.from_numpy(b))
+    return d, offs
+
+
+def _time_launches(torch, fn, steps, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _record(name, recs, ms_per_call, n_calls_bytes, peak, extra=None):
+    n = sum(r["n"] for r in recs)
+    blob = sum(int(r["blob"].size) for r in recs)
+    hist = sum(r["hist"].astype(np.float64) for r in recs)
+    code_bits = sum(int(r["info"].code_bits) for r in recs)
+    alg = blob + n
+    d = {"workload": name, "tensors": len(recs), "n_bytes": n, "compressed_bytes": blob,
+         "ratio": round(n / blob, 4), "savings_pct": round(100 * (1 - blob / n), 2),
+         "exponent_entropy_bits": round(entropy_bits(hist), 4), "mean_code_bits": round(code_bits / n, 4),
+         "codes_le6_bits_frac": round(sum(r["le6"] * r["n"] for r in recs) / n, 5),
+         "max_code_bits": max(int(r["info"].max_len) for r in recs),
+         "ms_per_call": round(ms_per_call, 5), "gbps_fp8_out": round(n_calls_bytes / ms_per_call / 1e6, 2),
+         "roofline_frac": round(alg / ms_per_call / 1e6 / peak, 4) if extra is None or "alg_bytes" not in extra
+         else round(extra["alg_bytes"] / ms_per_call / 1e6 / peak, 4)}
+    if extra:
+        d.update({k: v for k, v in extra.items() if k != "alg_bytes"})
+    print(json.dumps(d), flush=True)
+    return d
+
+
+def run_sweep(args):
+    """Every workload: compression ratio, exponent entropy, decode GB/s and
+    roofline fraction, each output checked byte for byte against its source."""
+    import torch
+    L = load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, _ = measured_hbm_peak()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    results = []
+    names = args.sweep.split(",") if args.sweep != "all" else ["single_1k", "llama3_8b_layer", "sweep", "moe",
+                                                                  "llama3_70b"]
+
+    def check_outputs(recs, d_out, out_offs):
+        assert int(status.item()) == 0, f"decode status {int(status.item())}"
+        for r, o in zip(recs, out_offs):
+            got = d_out[o:o + r["n"]].cpu().numpy()
+            assert _blake(got) == r["hash"], f"{r['name']}: decoded bytes differ from the source"
+
+    def batched(recs, steps, name, extra=None):
+        d_blob, offs = _upload(torch, dev, [r["blob"] for r in recs])
+        out_offs, o = [], 0
+        for r in recs:
+            out_offs.append(o)
+            o += (r["n"] + 255) // 256 * 256
+        d_out = torch.empty(o, dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(L.batched_workspace_size(len(recs)), 16), dtype=torch.uint8, device=dev)
+        batch = L.make_batch([L.BatchItem(r["info"], int(d_blob.data_ptr()) + bo, int(d_out.data_ptr()) + oo)
+                              for r, bo, oo in zip(recs, offs, out_offs)])
+        fn = lambda: L.decode_batched(batch, workspace=ws, status=status)  # noqa: E731
+        ms = _time_launches(torch, fn, steps, 3)
+        check_outputs(recs, d_out, out_offs)
+        n = sum(r["n"] for r in recs)
+        res = _record(name, recs, ms, n, peak, extra)
+        del d_blob, d_out
+        torch.cuda.empty_cache()
+        return res
+
+    for nm in names:
+        if nm == "single_1k":
+            recs = _encode_specs(synth.single_normal_1k().tensors, L)
+            d_blob, _ = _upload(torch, dev, [recs[0]["blob"]])
+            d_out = torch.empty(recs[0]["n"], dtype=torch.uint8, device=dev)
+            fn = lambda: L.decode(recs[0]["info"], d_blob, d_out, status=status)  # noqa: E731
+            ms = _time_launches(torch, fn, args.steps, 3)
+            check_outputs(recs, d_out, [0])
+            results.append(_record("single_1024x1024_normal16", recs, ms, recs[0]["n"], peak,
+                                   {"launch": "ecf8_decode", "l2": "fits in L2"}))
+        elif nm == "llama3_8b_layer":
+            recs = _encode_specs(synth.llama3_8b_layer().tensors, L)
+            results.append(batched(recs, args.steps, "llama3_8b_layer_sas1.8", {"launch": "ecf8_decode_batched"}))
+        elif nm == "sweep":
+            for a in synth.SWEEP_ALPHAS:
+                for m in synth.SWEEP_MAXES:
+                    wl = synth.alpha_sweep_point(a, m)
+                    recs = _encode_specs(wl.tensors, L)
+                    d_blob, _ = _upload(torch, dev, [recs[0]["blob"]])
+                    d_out = torch.empty(recs[0]["n"], dtype=torch.uint8, device=dev)
+                    fn = lambda: L.decode(recs[0]["info"], d_blob, d_out, status=status)  # noqa: E731
+                    ms = _time_launches(torch, fn, args.steps, 3)
+                    check_outputs(recs, d_out, [0])
+                    results.append(_record(wl.name, recs, ms, recs[0]["n"], peak,
+                                           {"launch": "ecf8_decode", "alpha": a, "max_abs": m}))
+                    del d_blob, d_out
+        elif nm == "moe":
+            wl = synth.moe_experts(args.moe_experts)
+            recs = _encode_specs(wl.tensors, L)
+            results.append(batched(recs, max(3, args.steps // 20), wl.name,
+                                   {"launch": "ecf8_decode_batched (workspace)"}))
+        elif nm == "llama3_70b":
+            # layer 0 is generated; layers 1..79 are device copies of its blobs
+            # (host generation of all 68.45e9 weights would take ~30 min), so the
+            # loop walks ~54 GB of distinct resident compressed bytes
+            recs = _encode_specs(synth.llama3_70b_layer(0).tensors, L)
+            layers = args.layers
+            d_blob, offs = _upload(torch, dev, [r["blob"] for r in recs])
+            copies = [d_blob] + [d_blob.clone() for _ in range(layers - 1)]
+            out_offs, o = [], 0
+            for r in recs:
+                out_offs.append(o)
+                o += (r["n"] + 255) // 256 * 256
+            d_out = torch.empty(o, dtype=torch.uint8, device=dev)  # one buffer reused by every layer
+            batches = [L.make_batch([L.BatchItem(r["info"], int(c.data_ptr()) + bo, int(d_out.data_ptr()) + oo)
+                                     for r, bo, oo in zip(recs, offs, out_offs)]) for c in copies]
+
+            def all_layers():
+                for b in batches:
+                    L.decode_batched(b, status=status)
+
+            ms = _time_launches(torch, all_layers, max(1, args.steps // 50), 1)
+            check_outputs(recs, d_out, out_offs)
+            n_layer = sum(r["n"] for r in recs)
+            blob_layer = sum(int(r["blob"].size) for r in recs)
+            res = _record(f"llama3_70b_{layers}layers_reused_buffer", recs, ms, n_layer * layers, peak,
+                          {"launch": f"{layers} x ecf8_decode_batched into one reused buffer",
+                           "resident_compressed_bytes": blob_layer * layers,
+                           "alg_bytes": (blob_layer + n_layer) * layers,
+                           "note": "layers 1..N-1 are device copies of layer 0's blobs"})
+            results.append(res)
+            del copies, d_blob, d_out
+            torch.cuda.empty_cache()
+        else:
+            raise SystemExit(f"unknown sweep item {nm}")
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            for r in results:
+                f.write(json.dumps(r) + "\n")
+
+
 def load_library(build_only=False):
     from lossless_fp8_weight_b200 import _build
     _build.build()
@@ -281,12 +454,18 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--ref-sample", type=int, default=1 << 21)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", default=None, help="all, or a comma list of single_1k,llama3_8b_layer,sweep,moe,llama3_70b")
+    ap.add_argument("--sweep-out", default=None)
+    ap.add_argument("--moe-experts", type=int, default=256)
+    ap.add_argument("--layers", type=int, default=80)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     workload = workload_by_name(args.workload)
     if args.impl == "reference":
         return run_reference(args, workload)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch
     import torch.distributed as dist
