@@ -422,14 +422,36 @@ __device__ __forceinline__ int find_tensor(const DevTensor* ts, int count, uint3
   return lo;
 }
 
+// The group that starts at estimated cost c of the launch: in the tensor whose
+// cost range holds c, the first group whose cost range starts at or after c.
+// Non-decreasing in c, 0 at c = 0 and the launch's group count at its total
+// cost, so consecutive cost cuts give disjoint group runs that cover all.
+__device__ __forceinline__ uint32_t group_at_cost(const DevTensor* ts, int count, uint64_t c) {
+  int lo = 0, hi = count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ts[mid].cost_base <= c) lo = mid;
+    else hi = mid - 1;
+  }
+  const uint64_t w = ts[lo].group_cost;
+  uint64_t k = (c - ts[lo].cost_base + w - 1) / w;
+  if (k > ts[lo].n_groups) k = ts[lo].n_groups;
+  return ts[lo].group_base + (uint32_t)k;
+}
+
 // Persistent CTA over a contiguous run of groups (across tensors, in table
-// order).  Within each tensor's part of the run, warp w takes groups w, w+W,
-// ... and fetches its next group while decoding the current one.
-__device__ __forceinline__ void decode_run(const DevTensor* table, int count, uint32_t total, int32_t* status) {
+// order) holding an equal share of the launch's estimated cost: a group of a
+// tensor with short codes holds more weights and takes longer.  Within each
+// tensor's part of the run, warp w takes groups w, w+W, ... and fetches its
+// next group while decoding the current one.
+__device__ __forceinline__ void decode_run(const DevTensor* table, int count, uint32_t total, uint64_t total_cost,
+                                           int32_t* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Smem* sm = reinterpret_cast<Smem*>(smem_raw);
-  const uint32_t gb = (uint32_t)((uint64_t)blockIdx.x * total / gridDim.x);
-  const uint32_t ge = (uint32_t)((uint64_t)(blockIdx.x + 1) * total / gridDim.x);
+  const uint32_t gb = group_at_cost(table, count, (uint64_t)blockIdx.x * total_cost / gridDim.x);
+  const uint32_t ge = blockIdx.x + 1 == gridDim.x
+                          ? total
+                          : group_at_cost(table, count, (uint64_t)(blockIdx.x + 1) * total_cost / gridDim.x);
   if (gb >= ge) return;
   const uint32_t warp = threadIdx.x >> 5;
   WarpArea* wa = &sm->warp[warp];
@@ -458,8 +480,9 @@ __device__ __forceinline__ void decode_run(const DevTensor* table, int count, ui
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_table_kernel(const DevTensor* __restrict__ ts, int count,
-                                                                    uint32_t total, int32_t* status) {
-  decode_run(ts, count, total, status);
+                                                                    uint32_t total, uint64_t total_cost,
+                                                                    int32_t* status) {
+  decode_run(ts, count, total, total_cost, status);
 }
 
 // Small batches travel inside the launch's parameter block.
@@ -472,8 +495,9 @@ constexpr int kInlineMax = ECF8_BATCH_INLINE_MAX;
 
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1) decode_inline_kernel(const __grid_constant__ InlineBatch<N> b,
-                                                                     uint32_t total, int32_t* status) {
-  decode_run(b.t, b.count, total, status);
+                                                                     uint32_t total, uint64_t total_cost,
+                                                                     int32_t* status) {
+  decode_run(b.t, b.count, total, total_cost, status);
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -532,10 +556,23 @@ int check_info(const ecf8_info* info) {
   return ECF8_OK;
 }
 
+// Estimated cost of decoding one group of a tensor, in units of one decoded
+// weight: a fixed part (fetch, scan, table walk over the group's 1 KB of
+// code stream) worth about 2560 weights on B200, plus the weights the group
+// holds, which is 8192 bits over the mean code length.  Only the split of
+// work between CTAs depends on it, never the bytes decoded.
+constexpr uint32_t kGroupFixedCost = 2560;
+uint32_t group_cost(const ecf8_info* info) {
+  const uint64_t bits = (uint64_t)kC * kT * 8;
+  uint64_t codes = info->code_bits ? bits * info->n / info->code_bits : bits;
+  if (codes > bits) codes = bits;
+  return kGroupFixedCost + (uint32_t)codes;
+}
+
 DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
   const uint8_t* b = static_cast<const uint8_t*>(d_blob);
   DevTensor t;
-  t.lut = reinterpret_cast<const uint32_t*>(b + info->lut_off);
+  t.cost_base = 0;
   t.gaps = reinterpret_cast<const uint32_t*>(b + info->gaps_off);
   t.groups = reinterpret_cast<const uint64_t*>(b + info->groups_off);
   t.stream = reinterpret_cast<const uint32_t*>(b + info->stream_off);
@@ -545,24 +582,51 @@ DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
   t.code_bits = info->code_bits;
   t.n_groups = info->n_groups;
   t.group_base = 0;
+  t.group_cost = group_cost(info);
   for (int s = 0; s < 16; ++s) t.len[s] = info->len[s];
   return t;
 }
 
-// Checks one tensor of a call and appends its descriptor (skipping n = 0).
-int add_tensor(const ecf8_info* info, const void* d_blob, uint8_t* d_out, std::vector<DevTensor>& v,
-               uint64_t& groups) {
-  int rc = check_info(info);
-  if (rc) return rc;
-  if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
-  if (info->n == 0) return ECF8_OK;
-  if (!d_blob || !d_out) return ECF8_ERR_ARG;
-  if (!aligned16(d_blob) || !aligned16(d_out)) return ECF8_ERR_ALIGN;
-  DevTensor t = make_dev(info, d_blob, d_out);
+// Appends a checked descriptor to a launch: its group and cost offsets.
+int append(DevTensor t, DevTensor* table, size_t at, uint64_t& groups, uint64_t& cost) {
   t.group_base = (uint32_t)groups;
-  groups += info->n_groups;
+  t.cost_base = cost;
+  groups += t.n_groups;
+  cost += (uint64_t)t.n_groups * t.group_cost;
   if (groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
-  v.push_back(t);
+  table[at] = t;
+  return ECF8_OK;
+}
+
+// Checks one tensor of a call; *skip is set for an empty tensor (n = 0),
+// which the launch leaves out.
+int check_tensor(const ecf8_tensor& t, bool* skip) {
+  int rc = check_info(t.info);
+  if (rc) return rc;
+  if (t.info->chunk_bytes != (uint32_t)kC || t.info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
+  *skip = t.info->n == 0;
+  if (*skip) return ECF8_OK;
+  if (!t.d_blob || !t.d_out) return ECF8_ERR_ARG;
+  if (!aligned16(t.d_blob) || !aligned16(t.d_out)) return ECF8_ERR_ALIGN;
+  return ECF8_OK;
+}
+
+// Checks the tensors of a call and fills table[0, *used) with the descriptors
+// of the non-empty ones, with the launch's group count and total cost.
+int build_table(const ecf8_tensor* tensors, int count, DevTensor* table, int* used, uint64_t* groups,
+                uint64_t* cost) {
+  *used = 0;
+  *groups = *cost = 0;
+  for (int i = 0; i < count; ++i) {
+    bool skip = false;
+    int rc = check_tensor(tensors[i], &skip);
+    if (rc) return rc;
+    if (skip) continue;
+    rc = append(make_dev(tensors[i].info, tensors[i].d_blob, tensors[i].d_out), table, (size_t)*used, *groups,
+                *cost);
+    if (rc) return rc;
+    ++*used;
+  }
   return ECF8_OK;
 }
 
@@ -583,17 +647,15 @@ int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_
                 cudaStream_t s) {
   if (!info) return ECF8_ERR_ARG;
   if (n != info->n) return ECF8_ERR_ARG;
-  std::vector<DevTensor> v;
-  uint64_t groups = 0;
-  int rc = add_tensor(info, d_blob, d_out, v, groups);
-  if (rc || v.empty()) return rc;
+  ecf8_tensor one{info, d_blob, d_out};
+  InlineBatch<1> b;
+  uint64_t groups = 0, cost = 0;
+  int rc = build_table(&one, 1, b.t, &b.count, &groups, &cost);
+  if (rc || b.count == 0) return rc;
   uint32_t ctas = 0;
   if ((rc = grid_for_device(&ctas))) return rc;
-  InlineBatch<1> b;
-  b.t[0] = v[0];
-  b.count = 1;
-  decode_inline_kernel<1><<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(
-      b, (uint32_t)groups, d_status);
+  decode_inline_kernel<1><<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(b, (uint32_t)groups, cost,
+                                                                                    d_status);
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
   return ECF8_OK;
@@ -611,30 +673,25 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
     if (!d_workspace || workspace_bytes < ecf8_batched_workspace_size(count)) return ECF8_ERR_WORKSPACE;
     if (!aligned16(d_workspace)) return ECF8_ERR_ALIGN;
   }
-  std::vector<DevTensor> v;
-  v.reserve(count);
-  uint64_t groups = 0;
-  for (int i = 0; i < count; ++i) {
-    int rc = add_tensor(tensors[i].info, tensors[i].d_blob, tensors[i].d_out, v, groups);
-    if (rc) return rc;
-  }
-  if (v.empty()) return ECF8_OK;
+  std::vector<DevTensor> v((size_t)count);
+  int used = 0;
+  uint64_t groups = 0, cost = 0;
+  int rc = build_table(tensors, count, v.data(), &used, &groups, &cost);
+  if (rc || used == 0) return rc;
   uint32_t ctas = 0;
-  int rc = grid_for_device(&ctas);
-  if (rc) return rc;
+  if ((rc = grid_for_device(&ctas))) return rc;
   const uint32_t grid = grid_size(ctas, groups);
-  if (v.size() <= (size_t)kInlineMax) {
+  if (used <= kInlineMax) {
     InlineBatch<kInlineMax> b;
-    for (size_t i = 0; i < v.size(); ++i) b.t[i] = v[i];
-    b.count = (int)v.size();
-    decode_inline_kernel<kInlineMax><<<grid, kThreads, sizeof(Smem), s>>>(b, (uint32_t)groups,
-                                                                                          d_status);
+    for (int i = 0; i < used; ++i) b.t[i] = v[i];
+    b.count = used;
+    decode_inline_kernel<kInlineMax><<<grid, kThreads, sizeof(Smem), s>>>(b, (uint32_t)groups, cost, d_status);
   } else {
-    if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * v.size(), cudaMemcpyHostToDevice, s) !=
+    if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * (size_t)used, cudaMemcpyHostToDevice, s) !=
         cudaSuccess)
       return ECF8_ERR_CUDA;
-    decode_table_kernel<<<grid, kThreads, sizeof(Smem), s>>>(
-        static_cast<const DevTensor*>(d_workspace), (int)v.size(), (uint32_t)groups, d_status);
+    decode_table_kernel<<<grid, kThreads, sizeof(Smem), s>>>(static_cast<const DevTensor*>(d_workspace), used,
+                                                             (uint32_t)groups, cost, d_status);
   }
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -690,33 +747,19 @@ extern "C" int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count
   static std::mutex host_lock;
   std::lock_guard<std::mutex> guard(host_lock);
   int used = 0;
-  uint64_t groups = 0;
-  for (int i = 0; i < count; ++i) {
-    const ecf8_info* info = tensors[i].info;
-    int rc = check_info(info);
-    if (rc) return rc;
-    if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
-    if (info->n == 0) continue;
-    if (!tensors[i].d_blob || !tensors[i].d_out) return ECF8_ERR_ARG;
-    if (!aligned16(tensors[i].d_blob) || !aligned16(tensors[i].d_out)) return ECF8_ERR_ALIGN;
-    DevTensor t = make_dev(info, tensors[i].d_blob, tensors[i].d_out);
-    t.group_base = (uint32_t)groups;
-    groups += info->n_groups;
-    if (groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
-    host_table[used++] = t;
-  }
-  if (used == 0) return ECF8_OK;
+  uint64_t groups = 0, cost = 0;
+  int rc = build_table(tensors, count, host_table, &used, &groups, &cost);
+  if (rc || used == 0) return rc;
   DevTensor* table = nullptr;
-  int rc = noalloc_table_address(&table);
+  rc = noalloc_table_address(&table);
   if (rc) return rc;
   uint32_t ctas = 0;
   if ((rc = grid_for_device(&ctas))) return rc;
   if (cudaMemcpyAsync(table, host_table, sizeof(DevTensor) * (size_t)used, cudaMemcpyHostToDevice, s) !=
       cudaSuccess)
     return ECF8_ERR_CUDA;
-  decode_table_kernel<<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(table, used,
-                                                                                              (uint32_t)groups,
-                                                                                              d_status);
+  decode_table_kernel<<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(table, used, (uint32_t)groups, cost,
+                                                                              d_status);
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
   return ECF8_OK;

@@ -58,7 +58,7 @@ inline bool compute_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t 
 // What a decode kernel needs to know about one tensor, with device pointers
 // already resolved into the blob's sections.
 struct alignas(16) DevTensor {
-  const uint32_t* lut;
+  uint64_t cost_base;  // batched: estimated decode cost of all earlier tensors
   const uint32_t* gaps;
   const uint64_t* groups;
   const uint32_t* stream;
@@ -68,7 +68,9 @@ struct alignas(16) DevTensor {
   uint64_t code_bits;
   uint32_t n_groups;
   uint32_t group_base;  // batched: groups of all earlier tensors in the launch
+  uint32_t group_cost;  // estimated decode cost of one group of this tensor
   uint8_t len[16];
 };
+static_assert(sizeof(DevTensor) == 96, "descriptor size is part of the workspace contract");
 
 }  // namespace ecf8
