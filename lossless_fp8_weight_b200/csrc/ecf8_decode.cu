@@ -55,9 +55,11 @@ constexpr int kPadBits = 8 * kBytes;           // 272 bits walked by every lane
 constexpr int kPrivWords = kBytes + 1;         // parked exponent words per lane (<= 272 codes)
 constexpr int kMaxCodes = kSpanBits * kT;      // codes one group can hold: 8192
 constexpr int kStageWords = kMaxCodes / 8 + 8; // + alignment slack
+constexpr int kStagePhys = kStageWords + 2 * (kStageWords / 32 + 1) + 2;  // 2 pad words per 32
+
 constexpr int kWarps = 16;                     // warps per CTA
 constexpr int kThreads = 32 * kWarps;
-constexpr int kNU = 16;                        // 16-weight nibble units a lane prefetches in registers
+constexpr int kNU = 8;                         // 16-weight nibble units a lane prefetches in registers
 constexpr int kStates = 16;                    // tree nodes (<= 15 for 16 values) + the error state
 constexpr int kError = kStates - 1;
 
@@ -74,10 +76,15 @@ struct alignas(16) Tree {
 };
 struct alignas(16) WarpArea {
   uint32_t priv[kPrivWords * 32];  // word k of lane l at k*32 + l
-  uint32_t stage[kStageWords];     // read as uint4 per 32-weight block
+  uint32_t stage[kStagePhys];      // word w at sidx(w); read as uint2 per 16-weight unit
 };
 struct alignas(16) Smem {
-  uint2 fsm[kStates * 256];  // x: exponents (4 bits each, first lowest); y: byte0 next state, byte1 4*count
+  // the byte table, indexed by node << 8 | byte.  Wide entries (any code):
+  // x = exponents (4 bits each, first lowest), y = next node | 4*count << 8.
+  // Narrow entries (shortest code >= 2 bits, so <= 4 codes end in a byte;
+  // the first 16 KB): exponents in bits 0-15, next node in bits 16-23,
+  // 4*count in bits 24-31.
+  uint2 fsm[kStates * 256];
   Tree tree;
   WarpArea warp[kWarps];
 };
@@ -153,8 +160,14 @@ __device__ uint32_t bit_entry(const Tree* t, uint32_t state, uint32_t bit) {
   return t->ibase[l] + (v - t->first[l] - t->count[l]);
 }
 
+// Table widths: a tensor whose shortest code is 1 bit can end 8 codes in one
+// byte and needs the wide table; any other fits the narrow one, whose
+// lookups touch half the shared-memory banks of wide ones.
+constexpr int kWide = 64, kNarrow = 32;
+
 // K0: the tensor's tables into shared memory (all threads of the CTA):
 // bit steps -> 4-bit steps -> the byte table, each built from the last.
+template <int kW>
 __device__ void load_tables(const DevTensor* dt, Smem* sm) {
   Tree* t = &sm->tree;
   const int tid = threadIdx.x;
@@ -180,10 +193,25 @@ __device__ void load_tables(const DevTensor* dt, Smem* sm) {
     const uint32_t b = t->nib_step[(sa << 4) | (e & 15)];
     const uint32_t nb = (b >> 16) & 15u, sb = b >> 20;
     const uint32_t syms = (a & 0xFFFFu) | ((b & 0xFFFFu) << (4 * na));
-    sm->fsm[e] = sb == (uint32_t)kError ? make_uint2(0, kError) : make_uint2(syms, sb | ((4 * (na + nb)) << 8));
+    const uint32_t n4 = 4 * (na + nb);
+    if (kW == kWide)
+      sm->fsm[e] = sb == (uint32_t)kError ? make_uint2(0, kError) : make_uint2(syms, sb | (n4 << 8));
+    else
+      reinterpret_cast<uint32_t*>(sm->fsm)[e] = sb == (uint32_t)kError ? (uint32_t)kError << 16
+                                                                       : (syms & 0xFFFFu) | (sb << 16) | (n4 << 24);
   }
   __syncthreads();
 }
+
+// With the wide table, stage word w lives at w + 2*(w/32): when nearly every
+// code is 1 bit long, lanes' runs start 32 words apart and would otherwise
+// all store to one bank.  Word pairs (2u, 2u+1) stay adjacent and 8-byte
+// aligned.  With the narrow table (codes >= 2 bits) the plain layout spreads
+// the lanes' stores better.
+template <int kW>
+__device__ __forceinline__ uint32_t sidx(uint32_t w) { return kW == kWide ? w + ((w >> 5) << 1) : w; }
+template <int kW>  // uint2 index of unit u
+__device__ __forceinline__ uint32_t sunit(uint32_t u) { return kW == kWide ? u + (u >> 4) : u; }
 
 // ---------------------------------------------------------------- assembly
 
@@ -203,13 +231,14 @@ __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, 
 // A unit the group owns only in part (its first or last): lanes 0-15 write
 // one byte each, those inside [off0, off1).  `nw` is the unit's nibble word
 // holding this lane's weight (word (lane & 15) / 8), fetched at group start.
+template <int kW>
 __device__ __forceinline__ void ragged16(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1,
                                          const uint32_t* stage, uint32_t u, uint32_t nw) {
   const uint32_t lane = threadIdx.x & 31;
   const uint64_t p = gpos + lane;
   if (lane < 16 && p >= off0 && p < off1) {
     const uint32_t i = 16 * u + lane;
-    const uint32_t e = (stage[i >> 3] >> (4 * (i & 7))) & 15u;
+    const uint32_t e = (stage[sidx<kW>(i >> 3)] >> (4 * (i & 7))) & 15u;
     const uint32_t k = lane & 7;
     const uint32_t v = (nw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
     out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
@@ -248,6 +277,7 @@ __device__ __forceinline__ void fetch_group(const DevTensor* dt, uint32_t local,
   in.off1 = __ldg(dt->groups + local + 1);
 }
 
+template <int kW>
 __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t local, const GroupIn& in, Smem* sm,
                                               WarpArea* wa, int32_t* status) {
   const uint32_t lane = threadIdx.x & 31;
@@ -302,16 +332,27 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   // K2: the byte machine.  Every lane walks 272 bits; codes completed in the
   // zero bits after E are repeats of the all-zero code and are subtracted.
   uint32_t* priv = wa->priv + lane;
-  uint32_t y = 0;  // previous entry: byte0 = tree node (root), byte1 = 4 * codes
+  uint32_t y = 0;  // previous entry's node | count word (root, none)
   uint32_t acc = 0, sh = 0, words = 0;
 #pragma unroll
   for (int j = 0; j < kBytes; ++j) {
-    const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x7740u | (3u - (j & 3)));
-    const uint2 e = sm->fsm[idx];
-    y = e.y;
-    acc |= e.x << sh;
-    const uint32_t carry = __funnelshift_l(e.x, 0u, sh);
-    sh += e.y >> 8;
+    uint32_t x, n4;
+    if (kW == kWide) {
+      const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x7740u | (3u - (j & 3)));  // byte | node << 8
+      const uint2 e = sm->fsm[idx];
+      y = e.y;
+      x = e.x;
+      n4 = e.y >> 8;
+    } else {
+      const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x0060u | (3u - (j & 3))) & 0xFFFu;  // byte | node << 8
+      const uint32_t e = reinterpret_cast<const uint32_t*>(sm->fsm)[idx];
+      y = e;
+      x = e & 0xFFFFu;
+      n4 = e >> 24;
+    }
+    acc |= x << sh;
+    const uint32_t carry = __funnelshift_l(x, 0u, sh);
+    sh += n4;
     if (sh >= 32) {
       priv[32 * words] = acc;
       ++words;
@@ -322,8 +363,17 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   if (sh) priv[32 * words] = acc;
   const uint32_t emitted = 8 * words + sh / 4;
   const uint32_t extra = sm->tree.zero_codes[kPadBits - E];
-  const bool bad = (y & 0xFF) == (uint32_t)kError || emitted < extra;
+  const uint32_t node = kW == kWide ? y & 0xFFu : (y >> 16) & 0xFFu;
+  const bool bad = node == (uint32_t)kError || emitted < extra;
   const uint32_t cnt = bad ? 0 : emitted - extra;
+
+  // the rest of a group of many short codes, once the walk's registers are free
+  uint2 nv2[kNU];
+  if (units > 32u * kNU) {
+#pragma unroll
+    for (int j = 0; j < kNU; ++j)
+      if (lane + 32 * (kNU + j) < units) nv2[j] = __ldg(nib + lane + 32 * (kNU + j));
+  }
 
   // K3: place -- warp-shuffle scan of the counts
   uint32_t incl = cnt;
@@ -353,31 +403,28 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   const uint32_t q = (uint32_t)(off0 & 31) + start;
   const uint32_t d0 = q >> 3, dl = cnt ? (q + cnt - 1) >> 3 : 0;
   if (cnt) {
-    stage[d0] = 0;
-    stage[dl] = 0;
+    stage[sidx<kW>(d0)] = 0;
+    stage[sidx<kW>(dl)] = 0;
   }
   __syncwarp();
   if (cnt) {
     const uint32_t r = (q & 7) * 4;
     const uint32_t used = (cnt + 7) / 8;
     // the last parked word may hold padding codes after the lane's own ones
-    const uint32_t tail_mask = (cnt & 7) ? (1u << (4 * (cnt & 7))) - 1 : 0xFFFFFFFFu;
+    if (cnt & 7) priv[32 * (used - 1)] &= (1u << (4 * (cnt & 7))) - 1;
     const uint32_t nwd = dl - d0 + 1;  // destination words: used or used + 1
     uint32_t prev = priv[0];
-    if (used == 1) prev &= tail_mask;
-    atomicOr(&stage[d0], prev << r);
+    atomicOr(&stage[sidx<kW>(d0)], prev << r);
     uint32_t j = 1;
 #pragma unroll 4
     for (; j + 1 < nwd; ++j) {  // interior words belong to this lane alone
-      uint32_t cur = priv[32 * j];
-      if (j + 1 == used) cur &= tail_mask;
-      stage[d0 + j] = __funnelshift_l(prev, cur, r);
+      const uint32_t cur = priv[32 * j];
+      stage[sidx<kW>(d0 + j)] = __funnelshift_l(prev, cur, r);
       prev = cur;
     }
     if (nwd > 1) {
-      uint32_t cur = j < used ? priv[32 * j] : 0;
-      if (j + 1 == used) cur &= tail_mask;
-      atomicOr(&stage[d0 + j], __funnelshift_l(prev, cur, r));
+      const uint32_t cur = j < used ? priv[32 * j] : 0;
+      atomicOr(&stage[sidx<kW>(d0 + j)], __funnelshift_l(prev, cur, r));
     }
   }
   __syncwarp();
@@ -391,23 +438,36 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
 #pragma unroll
   for (int j = 0; j < kNU; ++j) {
     const uint32_t u = lane + 32 * j;
-    if (u >= first_full && u < end_full) {
+    if (u < end_full && (j > 0 || u >= first_full)) {  // first_full <= 2
       uint32_t o[4];
-      const uint2 ex = st[u];
+      const uint2 ex = st[sunit<kW>(u)];
       assemble8(ex.x, nv[j].x, o[0], o[1]);
       assemble8(ex.y, nv[j].y, o[2], o[3]);
       *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-  for (uint32_t u = lane + 32 * kNU; u < end_full; u += 32) {
+  if (end_full > 32u * kNU) {
+#pragma unroll
+    for (int j = 0; j < kNU; ++j) {
+      const uint32_t u = lane + 32 * (kNU + j);
+      if (u < end_full) {
+        uint32_t o[4];
+        const uint2 ex = st[sunit<kW>(u)];
+        assemble8(ex.x, nv2[j].x, o[0], o[1]);
+        assemble8(ex.y, nv2[j].y, o[2], o[3]);
+        *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+  for (uint32_t u = lane + 64 * kNU; u < end_full; u += 32) {
     uint32_t o[4];
-    const uint2 ex = st[u], nb = __ldg(nib + u);
+    const uint2 ex = st[sunit<kW>(u)], nb = __ldg(nib + u);
     assemble8(ex.x, nb.x, o[0], o[1]);
     assemble8(ex.y, nb.y, o[2], o[3]);
     *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  if (hr) ragged16(out, base + 16ull * u0, off0, off1, stage, u0, head_w);
-  if (tr) ragged16(out, base + 16ull * end_full, off0, off1, stage, end_full, tail_w);
+  if (hr) ragged16<kW>(out, base + 16ull * u0, off0, off1, stage, u0, head_w);
+  if (tr) ragged16<kW>(out, base + 16ull * end_full, off0, off1, stage, end_full, tail_w);
   __syncwarp();  // the stage and private words are reused by this warp's next group
 }
 
@@ -444,14 +504,14 @@ __device__ __forceinline__ uint32_t group_at_cost(const DevTensor* ts, int count
 // tensor with short codes holds more weights and takes longer.  Within each
 // tensor's part of the run, warp w takes groups w, w+W, ... and fetches its
 // next group while decoding the current one.
+template <int kW>
 __device__ __forceinline__ void decode_run(const DevTensor* table, int count, uint32_t total, uint64_t total_cost,
-                                           int32_t* status) {
+                                           uint32_t cta, uint32_t ctas, int32_t* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Smem* sm = reinterpret_cast<Smem*>(smem_raw);
-  const uint32_t gb = group_at_cost(table, count, (uint64_t)blockIdx.x * total_cost / gridDim.x);
-  const uint32_t ge = blockIdx.x + 1 == gridDim.x
-                          ? total
-                          : group_at_cost(table, count, (uint64_t)(blockIdx.x + 1) * total_cost / gridDim.x);
+  const uint32_t gb = group_at_cost(table, count, (uint64_t)cta * total_cost / ctas);
+  const uint32_t ge =
+      cta + 1 == ctas ? total : group_at_cost(table, count, (uint64_t)(cta + 1) * total_cost / ctas);
   if (gb >= ge) return;
   const uint32_t warp = threadIdx.x >> 5;
   WarpArea* wa = &sm->warp[warp];
@@ -461,7 +521,7 @@ __device__ __forceinline__ void decode_run(const DevTensor* table, int count, ui
     const DevTensor* dt = table + ti;
     const uint32_t tb = dt->group_base, te = tb + dt->n_groups;
     const uint32_t g1 = te < ge ? te : ge;  // this tensor's part of the run: [g0, g1)
-    load_tables(dt, sm);
+    load_tables<kW>(dt, sm);
     uint32_t g = g0 + warp;
     if (g < g1) {
       GroupIn in;
@@ -470,7 +530,7 @@ __device__ __forceinline__ void decode_run(const DevTensor* table, int count, ui
         GroupIn nx;
         const bool more = g + kWarps < g1;
         if (more) fetch_group(dt, g + kWarps - tb, nx);
-        process_group(dt, g - tb, in, sm, wa, status);
+        process_group<kW>(dt, g - tb, in, sm, wa, status);
         if (more) in = nx;
       }
     }
@@ -479,25 +539,49 @@ __device__ __forceinline__ void decode_run(const DevTensor* table, int count, ui
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_table_kernel(const DevTensor* __restrict__ ts, int count,
-                                                                    uint32_t total, uint64_t total_cost,
+// The two parts of a launch: the tensors that need the wide table come
+// first in the descriptor table and are decoded by CTAs [0, split); the
+// others, from descriptor `first` on, by CTAs [split, grid).  Each part
+// spreads its own estimated cost evenly over its CTAs.  The branch on the
+// part is taken once per CTA, so each part's code keeps its own registers.
+struct PartArgs {
+  int first, count;
+  uint32_t groups;
+  uint64_t cost;
+};
+struct SplitArgs {
+  uint32_t split;
+  PartArgs part[2];
+};
+
+__device__ __forceinline__ void decode_split(const DevTensor* t, const SplitArgs& a, int32_t* status) {
+  if (blockIdx.x < a.split) {
+    const PartArgs& p = a.part[0];
+    decode_run<kWide>(t + p.first, p.count, p.groups, p.cost, blockIdx.x, a.split, status);
+  } else {
+    const PartArgs& p = a.part[1];
+    decode_run<kNarrow>(t + p.first, p.count, p.groups, p.cost, blockIdx.x - a.split, gridDim.x - a.split, status);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_table_kernel(const DevTensor* __restrict__ ts,
+                                                                    const __grid_constant__ SplitArgs a,
                                                                     int32_t* status) {
-  decode_run(ts, count, total, total_cost, status);
+  decode_split(ts, a, status);
 }
 
 // Small batches travel inside the launch's parameter block.
 template <int N>
 struct InlineBatch {
   DevTensor t[N];
-  int count;
 };
 constexpr int kInlineMax = ECF8_BATCH_INLINE_MAX;
 
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1) decode_inline_kernel(const __grid_constant__ InlineBatch<N> b,
-                                                                     uint32_t total, uint64_t total_cost,
+                                                                     const __grid_constant__ SplitArgs a,
                                                                      int32_t* status) {
-  decode_run(b.t, b.count, total, total_cost, status);
+  decode_split(b.t, a, status);
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -515,9 +599,9 @@ int grid_for_device(uint32_t* ctas) {
     return ECF8_OK;
   }
   const int bytes = (int)sizeof(Smem);
-  if (cudaFuncSetAttribute(decode_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
-      cudaFuncSetAttribute(decode_inline_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ||
-      cudaFuncSetAttribute(decode_inline_kernel<kInlineMax>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))
+  const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if (cudaFuncSetAttribute(decode_table_kernel, a, bytes) || cudaFuncSetAttribute(decode_inline_kernel<1>, a, bytes) ||
+      cudaFuncSetAttribute(decode_inline_kernel<kInlineMax>, a, bytes))
     return ECF8_ERR_CUDA;
   int sms = 0, per_sm = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
@@ -556,17 +640,24 @@ int check_info(const ecf8_info* info) {
   return ECF8_OK;
 }
 
+// The table width a tensor needs: wide when some code is 1 bit long.
+int width_of(const ecf8_info* info) {
+  for (int v = 0; v < 16; ++v)
+    if (info->len[v] == 1) return kWide;
+  return kNarrow;
+}
+
 // Estimated cost of decoding one group of a tensor, in units of one decoded
 // weight: a fixed part (fetch, scan, table walk over the group's 1 KB of
-// code stream) worth about 2560 weights on B200, plus the weights the group
-// holds, which is 8192 bits over the mean code length.  Only the split of
-// work between CTAs depends on it, never the bytes decoded.
-constexpr uint32_t kGroupFixedCost = 2560;
+// code stream), worth about 2560 weights on B200 with the wide table and
+// 1800 with the narrow one, plus the weights the group holds, which is 8192
+// bits over the mean code length.  Only the split of work between CTAs
+// depends on it, never the bytes decoded.
 uint32_t group_cost(const ecf8_info* info) {
   const uint64_t bits = (uint64_t)kC * kT * 8;
   uint64_t codes = info->code_bits ? bits * info->n / info->code_bits : bits;
   if (codes > bits) codes = bits;
-  return kGroupFixedCost + (uint32_t)codes;
+  return (width_of(info) == kWide ? 2560u : 1800u) + (uint32_t)codes;
 }
 
 DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
@@ -587,17 +678,6 @@ DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
   return t;
 }
 
-// Appends a checked descriptor to a launch: its group and cost offsets.
-int append(DevTensor t, DevTensor* table, size_t at, uint64_t& groups, uint64_t& cost) {
-  t.group_base = (uint32_t)groups;
-  t.cost_base = cost;
-  groups += t.n_groups;
-  cost += (uint64_t)t.n_groups * t.group_cost;
-  if (groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
-  table[at] = t;
-  return ECF8_OK;
-}
-
 // Checks one tensor of a call; *skip is set for an empty tensor (n = 0),
 // which the launch leaves out.
 int check_tensor(const ecf8_tensor& t, bool* skip) {
@@ -611,26 +691,81 @@ int check_tensor(const ecf8_tensor& t, bool* skip) {
   return ECF8_OK;
 }
 
-// Checks the tensors of a call and fills table[0, *used) with the descriptors
-// of the non-empty ones, with the launch's group count and total cost.
-int build_table(const ecf8_tensor* tensors, int count, DevTensor* table, int* used, uint64_t* groups,
-                uint64_t* cost) {
-  *used = 0;
-  *groups = *cost = 0;
+// The descriptors of one launch: table[first, first + count), with the
+// launch's group count and total estimated cost.
+struct Part {
+  int first = 0, count = 0;
+  uint64_t groups = 0, cost = 0;
+};
+
+// Checks the tensors of a call and fills table[] with the descriptors of the
+// non-empty ones: the wide-table ones first (part[0]), then the narrow ones
+// (part[1]), each part with its own group and cost offsets.
+int build_table(const ecf8_tensor* tensors, int count, DevTensor* table, Part part[2]) {
+  part[0] = part[1] = Part();
   for (int i = 0; i < count; ++i) {
     bool skip = false;
     int rc = check_tensor(tensors[i], &skip);
     if (rc) return rc;
-    if (skip) continue;
-    rc = append(make_dev(tensors[i].info, tensors[i].d_blob, tensors[i].d_out), table, (size_t)*used, *groups,
-                *cost);
-    if (rc) return rc;
-    ++*used;
+    if (!skip) part[width_of(tensors[i].info) == kWide ? 0 : 1].count++;
+  }
+  part[1].first = part[0].count;
+  int at[2] = {0, part[1].first};
+  for (int i = 0; i < count; ++i) {
+    const ecf8_info* info = tensors[i].info;
+    if (info->n == 0) continue;
+    const int k = width_of(info) == kWide ? 0 : 1;
+    DevTensor t = make_dev(info, tensors[i].d_blob, tensors[i].d_out);
+    t.group_base = (uint32_t)part[k].groups;
+    t.cost_base = part[k].cost;
+    part[k].groups += t.n_groups;
+    part[k].cost += (uint64_t)t.n_groups * t.group_cost;
+    if (part[k].groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
+    table[at[k]++] = t;
   }
   return ECF8_OK;
 }
 
-uint32_t grid_size(uint32_t ctas, uint64_t groups) { return (uint32_t)(groups < ctas ? groups : ctas); }
+// One launch for both parts: the grid is split between them in proportion
+// to their estimated cost.  Descriptors travel in the parameter block (h,
+// when d_table is null) or are read from d_table (device, already filled).
+int launch_parts(const DevTensor* h, const DevTensor* d_table, const Part part[2], int32_t* status,
+                 cudaStream_t s) {
+  const uint64_t groups = part[0].groups + part[1].groups;
+  if (groups == 0) return ECF8_OK;
+  uint32_t ctas = 0;
+  int rc = grid_for_device(&ctas);
+  if (rc) return rc;
+  const uint32_t grid = (uint32_t)(groups < ctas ? groups : ctas);
+  SplitArgs a;
+  for (int k = 0; k < 2; ++k) a.part[k] = PartArgs{part[k].first, part[k].count, (uint32_t)part[k].groups, part[k].cost};
+  if (part[0].groups == 0) {
+    a.split = 0;
+  } else if (part[1].groups == 0) {
+    a.split = grid;
+  } else {
+    const double f = (double)part[0].cost / (double)(part[0].cost + part[1].cost);
+    uint32_t sp = (uint32_t)(f * grid + 0.5);
+    sp = sp < 1 ? 1 : sp > grid - 1 ? grid - 1 : sp;
+    a.split = sp;
+  }
+  const int used = part[0].count + part[1].count;
+  if (d_table) {
+    decode_table_kernel<<<grid, kThreads, sizeof(Smem), s>>>(d_table, a, status);
+  } else if (used == 1) {
+    InlineBatch<1> b;
+    b.t[0] = h[0];
+    decode_inline_kernel<1><<<grid, kThreads, sizeof(Smem), s>>>(b, a, status);
+  } else {
+    if (used > kInlineMax) return ECF8_ERR_ARG;
+    InlineBatch<kInlineMax> b;
+    for (int i = 0; i < used; ++i) b.t[i] = h[i];
+    decode_inline_kernel<kInlineMax><<<grid, kThreads, sizeof(Smem), s>>>(b, a, status);
+  }
+  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ECF8_OK;
+}
 
 }  // namespace
 }  // namespace ecf8
@@ -647,18 +782,12 @@ int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_
                 cudaStream_t s) {
   if (!info) return ECF8_ERR_ARG;
   if (n != info->n) return ECF8_ERR_ARG;
-  ecf8_tensor one{info, d_blob, d_out};
-  InlineBatch<1> b;
-  uint64_t groups = 0, cost = 0;
-  int rc = build_table(&one, 1, b.t, &b.count, &groups, &cost);
-  if (rc || b.count == 0) return rc;
-  uint32_t ctas = 0;
-  if ((rc = grid_for_device(&ctas))) return rc;
-  decode_inline_kernel<1><<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(b, (uint32_t)groups, cost,
-                                                                                    d_status);
-  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
-  g_launches.fetch_add(1);
-  return ECF8_OK;
+  const ecf8_tensor one{info, d_blob, d_out};
+  DevTensor t[1];
+  Part part[2];
+  int rc = build_table(&one, 1, t, part);
+  if (rc) return rc;
+  return launch_parts(t, nullptr, part, d_status, s);
 }
 
 size_t ecf8_batched_workspace_size(int count) {
@@ -674,28 +803,18 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
     if (!aligned16(d_workspace)) return ECF8_ERR_ALIGN;
   }
   std::vector<DevTensor> v((size_t)count);
-  int used = 0;
-  uint64_t groups = 0, cost = 0;
-  int rc = build_table(tensors, count, v.data(), &used, &groups, &cost);
-  if (rc || used == 0) return rc;
-  uint32_t ctas = 0;
-  if ((rc = grid_for_device(&ctas))) return rc;
-  const uint32_t grid = grid_size(ctas, groups);
-  if (used <= kInlineMax) {
-    InlineBatch<kInlineMax> b;
-    for (int i = 0; i < used; ++i) b.t[i] = v[i];
-    b.count = used;
-    decode_inline_kernel<kInlineMax><<<grid, kThreads, sizeof(Smem), s>>>(b, (uint32_t)groups, cost, d_status);
-  } else {
-    if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * (size_t)used, cudaMemcpyHostToDevice, s) !=
-        cudaSuccess)
+  Part part[2];
+  int rc = build_table(tensors, count, v.data(), part);
+  if (rc) return rc;
+  const size_t used = (size_t)part[0].count + (size_t)part[1].count;
+  if (used == 0) return ECF8_OK;
+  const DevTensor* d_table = nullptr;
+  if (count > kInlineMax) {
+    if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * used, cudaMemcpyHostToDevice, s) != cudaSuccess)
       return ECF8_ERR_CUDA;
-    decode_table_kernel<<<grid, kThreads, sizeof(Smem), s>>>(static_cast<const DevTensor*>(d_workspace), used,
-                                                             (uint32_t)groups, cost, d_status);
+    d_table = static_cast<const DevTensor*>(d_workspace);
   }
-  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
-  g_launches.fetch_add(1);
-  return ECF8_OK;
+  return launch_parts(v.data(), d_table, part, d_status, s);
 }
 
 uint64_t ecf8_launch_count(void) { return g_launches.load(); }
@@ -746,21 +865,14 @@ extern "C" int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count
   static DevTensor host_table[ECF8_NOALLOC_MAX_TENSORS];
   static std::mutex host_lock;
   std::lock_guard<std::mutex> guard(host_lock);
-  int used = 0;
-  uint64_t groups = 0, cost = 0;
-  int rc = build_table(tensors, count, host_table, &used, &groups, &cost);
-  if (rc || used == 0) return rc;
-  DevTensor* table = nullptr;
-  rc = noalloc_table_address(&table);
+  Part part[2];
+  int rc = build_table(tensors, count, host_table, part);
   if (rc) return rc;
-  uint32_t ctas = 0;
-  if ((rc = grid_for_device(&ctas))) return rc;
-  if (cudaMemcpyAsync(table, host_table, sizeof(DevTensor) * (size_t)used, cudaMemcpyHostToDevice, s) !=
-      cudaSuccess)
+  const size_t used = (size_t)part[0].count + (size_t)part[1].count;
+  if (used == 0) return ECF8_OK;
+  DevTensor* table = nullptr;
+  if ((rc = noalloc_table_address(&table))) return rc;
+  if (cudaMemcpyAsync(table, host_table, sizeof(DevTensor) * used, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return ECF8_ERR_CUDA;
-  decode_table_kernel<<<grid_size(ctas, groups), kThreads, sizeof(Smem), s>>>(table, used, (uint32_t)groups, cost,
-                                                                              d_status);
-  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
-  g_launches.fetch_add(1);
-  return ECF8_OK;
+  return launch_parts(host_table, table, part, d_status, s);
 }
