@@ -51,6 +51,7 @@ constexpr int kC = 32, kT = 32;
 constexpr int kWords = kC / 4;                 // stream words per chunk
 constexpr int kSpanBits = 8 * kC;              // 256
 constexpr int kBytes = (kSpanBits + 15 + 7) / 8 + 0;  // 34: a lane may own up to 256 + 15 bits
+static_assert(kBytes % 2 == 0, "the narrow walk takes bytes in pairs");
 constexpr int kPadBits = 8 * kBytes;           // 272 bits walked by every lane
 constexpr int kPrivWords = kBytes + 1;         // parked exponent words per lane (<= 272 codes)
 constexpr int kMaxCodes = kSpanBits * kT;      // codes one group can hold: 8192
@@ -213,6 +214,15 @@ __device__ __forceinline__ uint32_t sidx(uint32_t w) { return kW == kWide ? w + 
 template <int kW>  // uint2 index of unit u
 __device__ __forceinline__ uint32_t sunit(uint32_t u) { return kW == kWide ? u + (u >> 4) : u; }
 
+// Index of a narrow-table entry: byte k of stream word w, then the node held
+// in byte 2 of entry e; the upper bytes replicate that byte's sign bit, which
+// is zero since nodes are < 16 (prmt's sign-replicate selector nibbles).
+__device__ __forceinline__ uint32_t nidx(uint32_t w, uint32_t e, uint32_t k) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(e), "r"(0xEE60u | k));
+  return r;
+}
+
 // ---------------------------------------------------------------- assembly
 
 __device__ __forceinline__ uint32_t bsel(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
@@ -334,30 +344,42 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   uint32_t* priv = wa->priv + lane;
   uint32_t y = 0;  // previous entry's node | count word (root, none)
   uint32_t acc = 0, sh = 0, words = 0;
+  if (kW == kWide) {
 #pragma unroll
-  for (int j = 0; j < kBytes; ++j) {
-    uint32_t x, n4;
-    if (kW == kWide) {
+    for (int j = 0; j < kBytes; ++j) {
       const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x7740u | (3u - (j & 3)));  // byte | node << 8
       const uint2 e = sm->fsm[idx];
       y = e.y;
-      x = e.x;
-      n4 = e.y >> 8;
-    } else {
-      const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x0060u | (3u - (j & 3))) & 0xFFFu;  // byte | node << 8
-      const uint32_t e = reinterpret_cast<const uint32_t*>(sm->fsm)[idx];
-      y = e;
-      x = e & 0xFFFFu;
-      n4 = e >> 24;
+      acc |= e.x << sh;
+      const uint32_t carry = __funnelshift_l(e.x, 0u, sh);
+      sh += e.y >> 8;
+      if (sh >= 32) {
+        priv[32 * words] = acc;
+        ++words;
+        acc = carry;
+        sh -= 32;
+      }
     }
-    acc |= x << sh;
-    const uint32_t carry = __funnelshift_l(x, 0u, sh);
-    sh += n4;
-    if (sh >= 32) {
-      priv[32 * words] = acc;
-      ++words;
-      acc = carry;
-      sh -= 32;
+  } else {
+    // two bytes per packing step: each ends at most 4 codes (16 bits), so a
+    // pair's exponents fit one word
+    const uint32_t* tab = reinterpret_cast<const uint32_t*>(sm->fsm);
+#pragma unroll
+    for (int j = 0; j < kBytes; j += 2) {
+      const uint32_t e1 = tab[nidx(sw[j >> 2], y, 3u - (j & 3))];
+      const uint32_t e2 = tab[nidx(sw[(j + 1) >> 2], e1, 3u - ((j + 1) & 3))];
+      y = e2;
+      const uint32_t n1 = e1 >> 24;
+      const uint32_t p = (e1 & 0xFFFFu) | ((e2 & 0xFFFFu) << n1);
+      acc |= p << sh;
+      const uint32_t carry = __funnelshift_l(p, 0u, sh);
+      sh += n1 + (e2 >> 24);
+      if (sh >= 32) {
+        priv[32 * words] = acc;
+        ++words;
+        acc = carry;
+        sh -= 32;
+      }
     }
   }
   if (sh) priv[32 * words] = acc;
