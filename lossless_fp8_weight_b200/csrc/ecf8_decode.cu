@@ -60,7 +60,7 @@ constexpr int kStagePhys = kStageWords + 2 * (kStageWords / 32 + 1) + 2;  // 2 p
 
 constexpr int kWarps = 16;                     // warps per CTA
 constexpr int kThreads = 32 * kWarps;
-constexpr int kNU = 8;                         // 16-weight nibble units a lane prefetches in registers
+constexpr int kND = 4;                         // 32-weight nibble blocks a lane prefetches in registers
 constexpr int kStates = 16;                    // tree nodes (<= 15 for 16 values) + the error state
 constexpr int kError = kStates - 1;
 
@@ -238,21 +238,31 @@ __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, 
   hi = __byte_perm(ev, od, 0x7362) | (n_hi & 0x87878787u);
 }
 
-// A unit the group owns only in part (its first or last): lanes 0-15 write
-// one byte each, those inside [off0, off1).  `nw` is the unit's nibble word
-// holding this lane's weight (word (lane & 15) / 8), fetched at group start.
-template <int kW>
-__device__ __forceinline__ void ragged16(uint8_t* out, uint64_t gpos, uint64_t off0, uint64_t off1,
-                                         const uint32_t* stage, uint32_t u, uint32_t nw) {
-  const uint32_t lane = threadIdx.x & 31;
-  const uint64_t p = gpos + lane;
-  if (lane < 16 && p >= off0 && p < off1) {
-    const uint32_t i = 16 * u + lane;
-    const uint32_t e = (stage[sidx<kW>(i >> 3)] >> (4 * (i & 7))) & 15u;
-    const uint32_t k = lane & 7;
-    const uint32_t v = (nw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
-    out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
+// 32 weights from their exponents (4 words, 8 per word) and nibbles (16
+// bytes), stored with one 32-byte store when the destination allows it.
+__device__ __forceinline__ void put32(uint8_t* dst, bool a32, uint4 ex, uint4 nb) {
+  uint32_t o[8];
+  assemble8(ex.x, nb.x, o[0], o[1]);
+  assemble8(ex.y, nb.y, o[2], o[3]);
+  assemble8(ex.z, nb.z, o[4], o[5]);
+  assemble8(ex.w, nb.w, o[6], o[7]);
+  if (a32) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(o[0]), "r"(o[1]),
+                 "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                 : "memory");
+  } else {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
+}
+
+// Exponents of the 32-weight block d (units 2d, 2d+1) from the stage.
+template <int kW>
+__device__ __forceinline__ uint4 stage32(const uint32_t* stage, uint32_t d) {
+  if (kW == kNarrow) return reinterpret_cast<const uint4*>(stage)[d];
+  const uint2* st = reinterpret_cast<const uint2*>(stage);
+  const uint2 a = st[sunit<kW>(2 * d)], b = st[sunit<kW>(2 * d + 1)];
+  return make_uint4(a.x, a.y, b.x, b.y);
 }
 
 // ---------------------------------------------------------------- one group per warp
@@ -300,19 +310,22 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   // base = off0 rounded down to 32); also the nibble words of the group's
   // first and last unit when the group owns them only in part
   const uint32_t units = offsets_ok ? (uint32_t)(((off0 & 31) + (off1 - off0) + 15) >> 4) : 0;
-  const uint2* nib = reinterpret_cast<const uint2*>(dt->nibbles) + (off0 >> 5) * 2;
-  uint2 nv[kNU];
+  const uint32_t blocks = (units + 1) >> 1;  // 32-weight blocks: 16 nibble bytes each
+  const uint4* nib = reinterpret_cast<const uint4*>(dt->nibbles) + (off0 >> 5);
+  uint4 nv[kND];
 #pragma unroll
-  for (int j = 0; j < kNU; ++j)
-    if (lane + 32 * j < units) nv[j] = __ldg(nib + lane + 32 * j);
+  for (int j = 0; j < kND; ++j)
+    if (lane + 32 * j < blocks) nv[j] = __ldg(nib + lane + 32 * j);
   const uint32_t* nib32 = reinterpret_cast<const uint32_t*>(nib);
   const uint32_t u0 = (uint32_t)(off0 & 31) >> 4;
   const uint32_t first_full = u0 + ((off0 & 15) ? 1u : 0u);
   const uint32_t end_full = (units && (off1 & 15)) ? units - 1 : units;
   const bool hr = units && first_full != u0;  // units == 0 when the offsets are not to be trusted
   const bool tr = end_full < units && !(hr && end_full == u0);
-  const uint32_t head_w = hr ? __ldg(nib32 + 2 * u0 + ((lane & 15) >> 3)) : 0u;
-  const uint32_t tail_w = tr ? __ldg(nib32 + 2 * end_full + ((lane & 15) >> 3)) : 0u;
+  // the ragged units' nibble words: lanes 0-15 the head's, lanes 16-31 the tail's
+  const bool rg = lane < 16 ? hr : tr;
+  const uint32_t ru = lane < 16 ? u0 : end_full;
+  const uint32_t rw = rg ? __ldg(nib32 + 2 * ru + ((lane & 15) >> 3)) : 0u;
 
   // K1: the lane's bits run from its first code (gap) to the next lane's
   // first code, or to the stream end: E bits once shifted to start at 0
@@ -390,11 +403,11 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   const uint32_t cnt = bad ? 0 : emitted - extra;
 
   // the rest of a group of many short codes, once the walk's registers are free
-  uint2 nv2[kNU];
-  if (units > 32u * kNU) {
+  uint4 nv2[kND];
+  if (kW == kWide && blocks > 32u * kND) {
 #pragma unroll
-    for (int j = 0; j < kNU; ++j)
-      if (lane + 32 * (kNU + j) < units) nv2[j] = __ldg(nib + lane + 32 * (kNU + j));
+    for (int j = 0; j < kND; ++j)
+      if (lane + 32 * (kND + j) < blocks) nv2[j] = __ldg(nib + lane + 32 * (kND + j));
   }
 
   // K3: place -- warp-shuffle scan of the counts
@@ -451,45 +464,53 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   }
   __syncwarp();
 
-  // K4b + K5: whole units by their lane -- consecutive lanes store
-  // consecutive 16 bytes, 512 contiguous bytes per instruction; the ragged
-  // first and last unit one byte per lane
+  // K4b + K5: whole 32-weight blocks by their lane -- consecutive lanes store
+  // consecutive 32 bytes, 1 KB contiguous per instruction; a whole unit
+  // whose block is not whole (at most one at each end) by lane 0 or 1; the
+  // ragged first and last unit one byte per lane
   const uint64_t base = off0 & ~31ull;
-  const uint2* st = reinterpret_cast<const uint2*>(stage);
   uint8_t* out = dt->out;
+  const bool a32 = ((reinterpret_cast<uintptr_t>(out) & 31) == 0);
 #pragma unroll
-  for (int j = 0; j < kNU; ++j) {
-    const uint32_t u = lane + 32 * j;
-    if (u < end_full && (j > 0 || u >= first_full)) {  // first_full <= 2
+  for (int j = 0; j < kND; ++j) {
+    const uint32_t d = lane + 32 * j;
+    if (2 * d + 2 <= end_full && (j > 0 || 2 * d >= first_full))  // first_full <= 2
+      put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv[j]);
+  }
+  if (kW == kWide && end_full > 64u * kND) {
+#pragma unroll
+    for (int j = 0; j < kND; ++j) {
+      const uint32_t d = lane + 32 * (kND + j);
+      if (2 * d + 2 <= end_full) put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv2[j]);
+    }
+  }
+  for (uint32_t d = lane + 32 * (kW == kWide ? 2 * kND : kND); 2 * d + 2 <= end_full; d += 32)
+    put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), __ldg(nib + d));
+  {
+    // a whole unit whose block partner is not whole: unit first_full when it
+    // is odd (lane 0), unit end_full - 1 when end_full is odd (lane 1)
+    uint32_t su = ~0u;
+    if (lane == 0 && (first_full & 1) && first_full < end_full) su = first_full;
+    if (lane == 1 && (end_full & 1) && end_full - 1 >= first_full) su = end_full - 1;
+    if (su != ~0u) {
+      const uint2 ex = reinterpret_cast<const uint2*>(stage)[sunit<kW>(su)];
+      const uint2 nb = reinterpret_cast<const uint2*>(nib)[su];
       uint32_t o[4];
-      const uint2 ex = st[sunit<kW>(u)];
-      assemble8(ex.x, nv[j].x, o[0], o[1]);
-      assemble8(ex.y, nv[j].y, o[2], o[3]);
-      *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
+      assemble8(ex.x, nb.x, o[0], o[1]);
+      assemble8(ex.y, nb.y, o[2], o[3]);
+      *reinterpret_cast<uint4*>(out + base + 16ull * su) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-  if (end_full > 32u * kNU) {
-#pragma unroll
-    for (int j = 0; j < kNU; ++j) {
-      const uint32_t u = lane + 32 * (kNU + j);
-      if (u < end_full) {
-        uint32_t o[4];
-        const uint2 ex = st[sunit<kW>(u)];
-        assemble8(ex.x, nv2[j].x, o[0], o[1]);
-        assemble8(ex.y, nv2[j].y, o[2], o[3]);
-        *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
+  if (hr || tr) {
+    const uint64_t p = base + 16ull * ru + (lane & 15);
+    if (rg && p >= off0 && p < off1) {
+      const uint32_t i = 16 * ru + (lane & 15);
+      const uint32_t e = (stage[sidx<kW>(i >> 3)] >> (4 * (i & 7))) & 15u;
+      const uint32_t k = lane & 7;
+      const uint32_t v = (rw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
+      out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
     }
   }
-  for (uint32_t u = lane + 64 * kNU; u < end_full; u += 32) {
-    uint32_t o[4];
-    const uint2 ex = st[sunit<kW>(u)], nb = __ldg(nib + u);
-    assemble8(ex.x, nb.x, o[0], o[1]);
-    assemble8(ex.y, nb.y, o[2], o[3]);
-    *reinterpret_cast<uint4*>(out + base + 16ull * u) = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-  if (hr) ragged16<kW>(out, base + 16ull * u0, off0, off1, stage, u0, head_w);
-  if (tr) ragged16<kW>(out, base + 16ull * end_full, off0, off1, stage, end_full, tail_w);
   __syncwarp();  // the stage and private words are reused by this warp's next group
 }
 
