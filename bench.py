@@ -437,6 +437,127 @@ def run_sweep(args):
                 f.write(json.dumps(r) + "\n")
 
 
+# Llama-3-8B layer tensors as (out_features, in_features) for y = x W^T
+_LAYER_SHAPES = {"q_proj": (4096, 4096), "k_proj": (1024, 4096), "v_proj": (1024, 4096), "o_proj": (4096, 4096),
+                 "gate_proj": (14336, 4096), "up_proj": (14336, 4096), "down_proj": (4096, 14336)}
+
+
+def run_pipeline(args):
+    """Decode-on-use (ECF8 walkthrough §3.2.2; DFloat11 article §4): a stack
+    of Llama-3-8B layers whose FP8 GEMMs (y = x W^T for all 7 projections, M
+    tokens) read weights that a 2-slot pool decodes one layer ahead on a
+    second stream.  Reports ms per layer for the GEMMs alone on resident
+    weights, decode then GEMMs on one stream, and the pipeline at several
+    decode grid caps, and checks every layer's GEMM outputs against the GEMMs
+    over the source weights."""
+    import torch
+    L = load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    recs = _encode_specs(synth.llama3_8b_layer().tensors, L, keep=True)
+    d_blob, offs = _upload(torch, dev, [r["blob"] for r in recs])
+    blobs = [d_blob[o:o + r["blob"].size] for r, o in zip(recs, offs)]
+    outs, o = [], 0
+    for r in recs:
+        outs.append(o)
+        o += (r["n"] + 255) // 256 * 256
+    slot_bytes = o
+    n_layers, M = args.pipeline_layers, args.pipeline_tokens
+    layers = [[L.PipelineTensor(r["info"], b, off) for r, b, off in zip(recs, blobs, outs)] for _ in range(n_layers)]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    one = torch.ones((), dtype=torch.float32, device=dev)
+    xs = {}
+    for r in recs:
+        k = _LAYER_SHAPES[r["name"]][1]
+        if k not in xs:
+            xs[k] = torch.from_numpy(synth.alpha_sweep_point(1.7, 448.0).tensors[0].generate(count=M * k)).to(
+                dev).view(torch.float8_e4m3fn).view(M, k)
+
+    def gemms(slot, ys=None):
+        for r, off in zip(recs, outs):
+            n_out, k = _LAYER_SHAPES[r["name"]]
+            w = slot[off:off + r["n"]].view(torch.float8_e4m3fn).view(n_out, k)
+            y = torch._scaled_mm(xs[k], w.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            if ys is not None:
+                ys.append(y)
+
+    # reference outputs: GEMMs over the source weights
+    ref = torch.empty(slot_bytes, dtype=torch.uint8, device=dev)
+    for r, off in zip(recs, outs):
+        ref[off:off + r["n"]].copy_(torch.from_numpy(r["x"]))
+    want = []
+    gemms(ref, want)
+    items = [L.BatchItem(r["info"], b, ref[off:off + r["n"]]) for r, b, off in zip(recs, blobs, outs)]
+    batch = L.make_batch(items)
+    reps = max(1, args.steps // 50)
+    results = {}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps / n_layers
+
+    results["gemm_only"] = timed(lambda: [gemms(ref) for _ in range(n_layers)])
+    results["decode_only"] = timed(lambda: [L.decode_batched(batch, status=status) for _ in range(n_layers)])
+
+    def serial():
+        for _ in range(n_layers):
+            L.decode_batched(batch, status=status)
+            gemms(ref)
+    results["serial"] = timed(serial)
+    assert int(status.item()) == 0
+
+    # the decode stream at high priority: its CTAs take SMs ahead of queued GEMM CTAs
+    compute, decode = torch.cuda.Stream(), torch.cuda.Stream(priority=-1)
+    slots = [torch.empty(slot_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    by_ptr = {t.data_ptr(): t for t in slots}
+    checked = False
+    for cap in args.pipeline_ctas:
+        P = L.Pipeline(layers, slots, slot_bytes, depth=1, max_ctas=cap, status=status, decode_stream=decode)
+
+        def one_pass(check=None):
+            for l in range(n_layers):
+                slot = by_ptr[P.acquire(l, compute)]
+                with torch.cuda.stream(compute):
+                    gemms(slot, check[l] if check is not None else None)
+                P.release(l, compute)
+
+        if not checked:
+            got = [[] for _ in range(n_layers)]
+            one_pass(got)
+            torch.cuda.synchronize()
+            for g in got:
+                assert all(torch.equal(a, b) for a, b in zip(g, want))
+            checked = True
+        one_pass()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(compute)
+        for _ in range(reps):
+            one_pass()
+        e1.record(compute)
+        torch.cuda.synchronize()
+        results[f"pipelined_ctas{cap}"] = e0.elapsed_time(e1) / reps / n_layers
+        P.close()
+    assert int(status.item()) == 0
+    best = min(v for k, v in results.items() if k.startswith("pipelined"))
+    hidden = (results["serial"] - best) / max(1e-9, results["serial"] - results["gemm_only"])
+    line = {"workload": f"pipeline_llama3_8b_x{n_layers}_tokens{M}", "metric": "ms per layer",
+            "gemm": "torch._scaled_mm e4m3 x e4m3 -> bf16, 7 projections",
+            "ms_per_layer": {k: round(v, 4) for k, v in results.items()},
+            "decode_hidden_frac": round(hidden, 3), "gemm_outputs_equal_source": True}
+    print(json.dumps(line), flush=True)
+    if args.sweep_out:
+        with open(args.sweep_out, "a") as f:
+            f.write(json.dumps(line) + "\n")
+
+
 def load_library(build_only=False):
     from lossless_fp8_weight_b200 import _build
     _build.build()
@@ -458,6 +579,10 @@ def main():
     ap.add_argument("--sweep-out", default=None)
     ap.add_argument("--moe-experts", type=int, default=256)
     ap.add_argument("--layers", type=int, default=80)
+    ap.add_argument("--pipeline", action="store_true", help="decode-on-use pipeline beside FP8 GEMMs")
+    ap.add_argument("--pipeline-layers", type=int, default=8)
+    ap.add_argument("--pipeline-tokens", type=int, default=2048)
+    ap.add_argument("--pipeline-ctas", type=lambda v: [int(c) for c in v.split(",")], default=[148, 74, 37, 18])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -466,6 +591,8 @@ def main():
         return run_reference(args, workload)
     if args.sweep:
         return run_sweep(args)
+    if args.pipeline:
+        return run_pipeline(args)
 
     import torch
     import torch.distributed as dist

@@ -188,6 +188,71 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
  *    nothing.  Other arguments and errors are as for ecf8_decode_batched. */
 int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count, int32_t* d_status, cudaStream_t s);
 
+/* ecf8_decode_batched with the persistent grid capped at max_ctas CTAs (one
+ * CTA occupies a whole SM's shared memory), so that a decode running beside
+ * other kernels leaves them the remaining SMs.  max_ctas = 0: one CTA per SM.
+ * A batch that mixes tensors with and without a 1-bit code takes at least 2. */
+int ecf8_decode_batched_ctas(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
+                             int32_t* d_status, cudaStream_t s, uint32_t max_ctas);
+
+/* ---------------------------------------------------------------------------
+ * Decode-on-use pipeline (ECF8 walkthrough §3.2.2 "即用即解压": a pool sized
+ * for the largest layer, the layer's forward pass triggers its decode, the
+ * pool is reused cyclically with no allocation; DFloat11 article §4: decode
+ * the next layers in the background while the current one computes).
+ *
+ * Layer m is decoded into slot m % n_slots on decode_stream, `depth` layers
+ * ahead of the one the compute stream asks for, once the compute stream has
+ * released that slot's previous layer.  Protocol per layer, in any order of
+ * layers (a forward pass takes them in order, and a new pass may start again
+ * at layer 0):
+ *     ecf8_pipeline_acquire(p, l, compute, &w);   -- compute waits for l
+ *     ... kernels on `compute` read layer l's FP8 weights at w ...
+ *     ecf8_pipeline_release(p, l, compute);       -- the slot may be reused
+ * n_slots must be at least depth + 1 (the slot being decoded ahead is never
+ * the one in use).  A layer still resident in its slot is not decoded again.
+ */
+typedef struct ecf8_layer_tensor {
+  const ecf8_info* info; /* host; copied at create time */
+  const void* d_blob;    /* device, 16-byte aligned, stays valid while the pipeline lives */
+  size_t out_offset;     /* byte offset of its FP8 output within a slot; multiple of 16 (of 32 for
+                            the fastest stores); out_offset + info->n <= slot_bytes */
+} ecf8_layer_tensor;
+
+typedef struct ecf8_layer {
+  const ecf8_layer_tensor* tensors; /* host; copied at create time */
+  int count;
+} ecf8_layer;
+
+typedef struct ecf8_pipeline ecf8_pipeline; /* opaque */
+
+/* Creates a pipeline over n_layers layers and n_slots caller-owned device
+ * buffers of slot_bytes each (16-byte aligned).  d_workspace (device) is
+ * needed only when a layer has more than ECF8_BATCH_INLINE_MAX tensors
+ * (ecf8_batched_workspace_size of the largest layer); d_status (device) gets
+ * the decodes' status bits.  max_ctas caps each decode's grid (0: one CTA
+ * per SM).  The pipeline creates two CUDA events per slot and allocates no
+ * device memory.  Errors: ECF8_ERR_ARG (counts, depth, slot too small),
+ * ECF8_ERR_ALIGN, ECF8_ERR_WORKSPACE, ECF8_ERR_CUDA. */
+int ecf8_pipeline_create(const ecf8_layer* layers, int n_layers, void* const* d_slots, int n_slots,
+                         size_t slot_bytes, int depth, uint32_t max_ctas, void* d_workspace,
+                         size_t workspace_bytes, int32_t* d_status, cudaStream_t decode_stream,
+                         ecf8_pipeline** out);
+
+/* Makes stream `compute` wait until layer's weights are decoded, enqueues the
+ * decodes of the next `depth` layers whose slots are free, and returns the
+ * layer's slot in *d_weights.  Returns ECF8_ERR_ARG if the layer's slot still
+ * holds another layer that has not been released. */
+int ecf8_pipeline_acquire(ecf8_pipeline* p, int layer, cudaStream_t compute, void** d_weights);
+
+/* Records, on `compute`, that the kernels reading layer's slot have been
+ * enqueued; a later decode into that slot waits for them. */
+int ecf8_pipeline_release(ecf8_pipeline* p, int layer, cudaStream_t compute);
+
+/* Frees the pipeline's events and host state (work already enqueued still
+ * runs to completion). */
+void ecf8_pipeline_destroy(ecf8_pipeline* p);
+
 /* Number of decode kernels this library has launched in this process. */
 uint64_t ecf8_launch_count(void);
 

@@ -91,6 +91,23 @@ _lib.ecf8_batched_workspace_size.argtypes = [_i32]
 _lib.ecf8_batched_workspace_size.restype = _sz
 _lib.ecf8_decode_batched.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p]
 _lib.ecf8_decode_batched_noalloc.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _p]
+_lib.ecf8_decode_batched_ctas.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p, _u32]
+
+
+class LayerTensor(ctypes.Structure):
+    _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("out_offset", ctypes.c_size_t)]
+
+
+class Layer(ctypes.Structure):
+    _fields_ = [("tensors", ctypes.POINTER(LayerTensor)), ("count", ctypes.c_int)]
+
+
+_lib.ecf8_pipeline_create.argtypes = [ctypes.POINTER(Layer), _i32, ctypes.POINTER(ctypes.c_void_p), _i32, _sz, _i32,
+                                      _u32, _p, _sz, _p, _p, ctypes.POINTER(ctypes.c_void_p)]
+_lib.ecf8_pipeline_acquire.argtypes = [_p, _i32, _p, ctypes.POINTER(ctypes.c_void_p)]
+_lib.ecf8_pipeline_release.argtypes = [_p, _i32, _p]
+_lib.ecf8_pipeline_destroy.argtypes = [_p]
+_lib.ecf8_pipeline_destroy.restype = None
 _lib.ecf8_launch_count.restype = ctypes.c_uint64
 _lib.ecf8_strerror.restype = ctypes.c_char_p
 _lib.ecf8_strerror.argtypes = [_i32]
@@ -214,9 +231,10 @@ def make_batch(items: Sequence[BatchItem]):
     return arr, keep
 
 
-def decode_batched(items, workspace=None, status=None, stream=None) -> None:
+def decode_batched(items, workspace=None, status=None, stream=None, max_ctas: int = 0) -> None:
     """Decode several blobs in one kernel launch.  ``items`` is a list of
-    BatchItem or the pair returned by make_batch."""
+    BatchItem or the pair returned by make_batch.  ``max_ctas`` > 0 caps the
+    persistent grid (one CTA per SM otherwise), leaving SMs to other kernels."""
     if isinstance(items, tuple):
         arr = items[0]
     else:
@@ -224,8 +242,12 @@ def decode_batched(items, workspace=None, status=None, stream=None) -> None:
     ws = _ptr(workspace)
     ws_bytes = int(workspace.numel() * workspace.element_size()) if workspace is not None and not isinstance(
         workspace, int) else 0
-    _check(_lib.ecf8_decode_batched(arr, len(arr), ws, ws_bytes, _ptr(status), _stream(stream)),
-           "ecf8_decode_batched")
+    if max_ctas:
+        _check(_lib.ecf8_decode_batched_ctas(arr, len(arr), ws, ws_bytes, _ptr(status), _stream(stream),
+                                             int(max_ctas)), "ecf8_decode_batched_ctas")
+    else:
+        _check(_lib.ecf8_decode_batched(arr, len(arr), ws, ws_bytes, _ptr(status), _stream(stream)),
+               "ecf8_decode_batched")
 
 
 def decode_batched_noalloc(items, status=None, stream=None) -> None:
@@ -240,3 +262,64 @@ def decode_batched_noalloc(items, status=None, stream=None) -> None:
         arr, _keep = make_batch(items)
     _check(_lib.ecf8_decode_batched_noalloc(arr, len(arr), _ptr(status), _stream(stream)),
            "ecf8_decode_batched_noalloc")
+
+
+@dataclass
+class PipelineTensor:
+    """One tensor of a pipeline layer: its blob info, device blob, and the
+    byte offset of its FP8 output inside a slot (multiple of 16)."""
+    info: Info
+    d_blob: object
+    out_offset: int
+
+
+class Pipeline:
+    """Decode-on-use over a fixed pool of slots (ecf8_pipeline_* in the C
+    ABI): layer m is decoded into slot m % len(slots) on ``decode_stream``,
+    ``depth`` layers ahead; ``acquire(l, stream)`` makes ``stream`` wait for
+    layer l and returns its slot, ``release(l, stream)`` lets the slot be
+    reused once the work already on ``stream`` is done."""
+
+    def __init__(self, layers, slots, slot_bytes: int, depth: int = 1, max_ctas: int = 0, workspace=None,
+                 status=None, decode_stream=None):
+        self._slots = list(slots)
+        self._keep = []
+        n = len(layers)
+        larr = (Layer * n)()
+        for l, tensors in enumerate(layers):
+            tarr = (LayerTensor * max(1, len(tensors)))()
+            for i, t in enumerate(tensors):
+                self._keep.append(t.info)
+                tarr[i].info = ctypes.pointer(t.info)
+                tarr[i].d_blob = _ptr(t.d_blob)
+                tarr[i].out_offset = int(t.out_offset)
+            self._keep.append(tarr)
+            larr[l].tensors = tarr
+            larr[l].count = len(tensors)
+        sarr = (ctypes.c_void_p * len(self._slots))(*[_ptr(x) for x in self._slots])
+        ws = _ptr(workspace)
+        ws_bytes = int(workspace.numel() * workspace.element_size()) if workspace is not None else 0
+        self._decode_stream = decode_stream
+        h = ctypes.c_void_p()
+        _check(_lib.ecf8_pipeline_create(larr, n, sarr, len(self._slots), int(slot_bytes), int(depth),
+                                         int(max_ctas), ws, ws_bytes, _ptr(status), _stream(decode_stream),
+                                         ctypes.byref(h)), "ecf8_pipeline_create")
+        self._h = h
+
+    def acquire(self, layer: int, stream=None) -> int:
+        """Device address of layer's slot; ``stream`` waits for its decode."""
+        w = ctypes.c_void_p()
+        _check(_lib.ecf8_pipeline_acquire(self._h, int(layer), _stream(stream), ctypes.byref(w)),
+               "ecf8_pipeline_acquire")
+        return int(w.value or 0)
+
+    def release(self, layer: int, stream=None) -> None:
+        _check(_lib.ecf8_pipeline_release(self._h, int(layer), _stream(stream)), "ecf8_pipeline_release")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.ecf8_pipeline_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()

@@ -773,13 +773,16 @@ int build_table(const ecf8_tensor* tensors, int count, DevTensor* table, Part pa
 // to their estimated cost.  Descriptors travel in the parameter block (h,
 // when d_table is null) or are read from d_table (device, already filled).
 int launch_parts(const DevTensor* h, const DevTensor* d_table, const Part part[2], int32_t* status,
-                 cudaStream_t s) {
+                 cudaStream_t s, uint32_t max_ctas = 0) {
   const uint64_t groups = part[0].groups + part[1].groups;
   if (groups == 0) return ECF8_OK;
   uint32_t ctas = 0;
   int rc = grid_for_device(&ctas);
   if (rc) return rc;
-  const uint32_t grid = (uint32_t)(groups < ctas ? groups : ctas);
+  if (max_ctas && max_ctas < ctas) ctas = max_ctas;
+  uint32_t grid = (uint32_t)(groups < ctas ? groups : ctas);
+  // a launch with both parts needs a CTA for each (a cap of 1 is raised to 2)
+  if (part[0].groups && part[1].groups && grid < 2) grid = 2;
   SplitArgs a;
   for (int k = 0; k < 2; ++k) a.part[k] = PartArgs{part[k].first, part[k].count, (uint32_t)part[k].groups, part[k].cost};
   if (part[0].groups == 0) {
@@ -837,8 +840,8 @@ size_t ecf8_batched_workspace_size(int count) {
   return count > kInlineMax ? sizeof(DevTensor) * (size_t)count : 0;
 }
 
-int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
-                        int32_t* d_status, cudaStream_t s) {
+int ecf8_decode_batched_ctas(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
+                             int32_t* d_status, cudaStream_t s, uint32_t max_ctas) {
   if (count < 0 || (count > 0 && !tensors)) return ECF8_ERR_ARG;
   if (count == 0) return ECF8_OK;
   if (count > kInlineMax) {
@@ -857,7 +860,12 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
       return ECF8_ERR_CUDA;
     d_table = static_cast<const DevTensor*>(d_workspace);
   }
-  return launch_parts(v.data(), d_table, part, d_status, s);
+  return launch_parts(v.data(), d_table, part, d_status, s, max_ctas);
+}
+
+int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
+                        int32_t* d_status, cudaStream_t s) {
+  return ecf8_decode_batched_ctas(tensors, count, d_workspace, workspace_bytes, d_status, s, 0);
 }
 
 uint64_t ecf8_launch_count(void) { return g_launches.load(); }
