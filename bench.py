@@ -664,21 +664,21 @@ def main():
     if world > 1:
         dist.barrier()
     launches0 = L.launch_count()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    # no events between the steps: each decode launch lets the next one start
+    # its prologue early (programmatic dependent launch), and an event in
+    # between would serialise them
     t0.record(stream)
     for k in range(args.steps):
-        ev[k][0].record(stream)
         step()
-        ev[k][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
     launches = L.launch_count() - launches0
     clk = clocks.stop()
     elapsed_ms = t0.elapsed_time(t1)
-    per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    per_launch_ms = elapsed_ms / max(1, launches)  # one decode launch per step
     elapsed_ms, per_launch_ms = max_over_ranks([elapsed_ms, per_launch_ms], dev)
     if world > 1:
         dist.barrier()

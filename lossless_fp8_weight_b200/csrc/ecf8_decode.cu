@@ -97,50 +97,72 @@ static_assert(sizeof(Smem) <= 227 * 1024, "shared memory budget");
 
 // ---------------------------------------------------------------- decode tables
 
-// Canonical code and internal-node numbering (one thread; a few hundred
-// instructions).  State 0 is the root; the internal nodes at depth l are the
-// values first[l] + count[l] + k, k < nint[l], numbered from ibase[l].
+// Canonical code and internal-node numbering, by one warp.  State 0 is the
+// root; the internal nodes at depth l are the values first[l] + count[l] + k,
+// k < nint[l], numbered from ibase[l].  Lane s < 16 holds symbol s's length;
+// lane l in 1..16 counts the codes of length l; a symbol's place in the
+// canonical order is its length's base plus its rank among the symbols of
+// that length.  Only the two 16-step recurrences (first codes, internal
+// nodes per depth) run on lane 0.
 __device__ void build_tree(const uint8_t* len, Tree* t) {
-  uint32_t count[17] = {};
-  uint32_t max_len = 0, present = 0;
-  uint64_t kraft = 0;
-  for (int s = 0; s < 16; ++s) {
-    const uint32_t l = len[s];
-    if (l) {
-      count[l]++;
-      present++;
-      kraft += 1ull << (16 - l);
-      max_len = l > max_len ? l : max_len;
-    }
-  }
-  uint32_t code = 0, base = 0, k = 0, lmin = 0;
-  for (int l = 1; l <= 16; ++l) {
-    code = (code + count[l - 1]) << 1;
-    t->first[l] = code;
-    t->count[l] = count[l];
-    t->base[l] = base;
-    base += count[l];
-    if (count[l] && !lmin) lmin = l;
-    for (int s = 0; s < 16; ++s)
-      if (len[s] == l) t->sorted[k++] = (uint8_t)s;
-  }
-  t->first[0] = t->count[0] = t->base[0] = 0;
-  int ok = present == 1 || kraft == (1ull << 16);
-  t->nint[0] = 1;
-  t->ibase[0] = 0;
-  uint32_t states = 1;
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t L = lane < 16 ? len[lane] : 0u;
+  uint32_t cnt = 0;
+#pragma unroll
   for (uint32_t l = 1; l <= 16; ++l) {
-    int64_t n = l < max_len ? 2 * (int64_t)t->nint[l - 1] - count[l] : 0;
-    if (n < 0) { ok = 0; n = 0; }
-    t->nint[l] = (uint32_t)n;
-    t->ibase[l] = states;
-    states += (uint32_t)n;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, L == l);
+    if (lane == l) cnt = __popc(m);
   }
-  if (states > kStates - 1) ok = 0;
-  t->nstates = states;
-  t->max_len = max_len;
-  t->ok = ok;
-  t->lmin = lmin ? lmin : 1;  // the all-zero path from the root meets a code after lmin zeros
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= (uint32_t)o) incl += v;
+  }
+  const uint32_t base = incl - cnt;  // lane l: codes shorter than l
+  const uint32_t my_base = __shfl_sync(0xFFFFFFFFu, base, L & 31u);
+  const uint32_t same = __match_any_sync(0xFFFFFFFFu, L);
+  const uint32_t rank = __popc(same & ((1u << lane) - 1u));
+  if (lane < 16 && L) t->sorted[my_base + rank] = (uint8_t)lane;
+  if (lane <= 16) {
+    t->count[lane] = cnt;
+    t->base[lane] = base;
+  }
+  const uint32_t max_len = __reduce_max_sync(0xFFFFFFFFu, L);
+  const uint32_t present = __popc(__ballot_sync(0xFFFFFFFFu, L != 0));
+  const uint32_t kraft = __reduce_add_sync(0xFFFFFFFFu, (L && L <= 16) ? 1u << (16 - L) : 0u);
+  const uint32_t lmin = __reduce_min_sync(0xFFFFFFFFu, L ? L : 99u);
+  __syncwarp();
+  if (lane == 0) {
+    uint32_t code = 0;
+    t->first[0] = 0;
+#pragma unroll
+    for (int l = 1; l <= 16; ++l) {
+      code = (code + t->count[l - 1]) << 1;
+      t->first[l] = code;
+    }
+    int ok = present == 1 || kraft == (1u << 16);
+    t->nint[0] = 1;
+    t->ibase[0] = 0;
+    uint32_t states = 1, prev = 1;
+#pragma unroll
+    for (uint32_t l = 1; l <= 16; ++l) {
+      int n = l < max_len ? 2 * (int)prev - (int)t->count[l] : 0;
+      if (n < 0) {
+        ok = 0;
+        n = 0;
+      }
+      t->nint[l] = (uint32_t)n;
+      t->ibase[l] = states;
+      states += (uint32_t)n;
+      prev = (uint32_t)n;
+    }
+    if (states > kStates - 1) ok = 0;
+    t->nstates = states;
+    t->max_len = max_len;
+    t->ok = ok;
+    t->lmin = lmin <= 16 ? lmin : 1;  // the all-zero path from the root meets a code after lmin zeros
+  }
 }
 
 // One bit from tree node `state`: the next node, and the value whose code
@@ -173,7 +195,7 @@ __device__ void load_tables(const DevTensor* dt, Smem* sm) {
   Tree* t = &sm->tree;
   const int tid = threadIdx.x;
   __syncthreads();  // every warp is done with the previous tensor's tables
-  if (tid == 0) build_tree(dt->len, t);
+  if (tid < 32) build_tree(dt->len, t);
   __syncthreads();
   if (tid < kStates * 2) t->bit_step[tid] = (uint16_t)bit_entry(t, tid >> 1, tid & 1);
   for (int z = tid; z <= kPadBits; z += kThreads) t->zero_codes[z] = (uint16_t)(z / t->lmin);
@@ -547,6 +569,13 @@ __device__ __forceinline__ uint32_t group_at_cost(const DevTensor* ts, int count
 // tensor with short codes holds more weights and takes longer.  Within each
 // tensor's part of the run, warp w takes groups w, w+W, ... and fetches its
 // next group while decoding the current one.
+// Programmatic dependent launch: the next kernel on the stream may start its
+// CTAs (on SMs this launch has left) before this grid ends; a decode builds
+// its first table from the codebook in its parameters before it waits for
+// the previous grid, whose writes it may read (blobs) or overwrite (outputs).
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <int kW>
 __device__ __forceinline__ void decode_run(const DevTensor* table, int count, uint32_t total, uint64_t total_cost,
                                            uint32_t cta, uint32_t ctas, int32_t* status) {
@@ -565,6 +594,7 @@ __device__ __forceinline__ void decode_run(const DevTensor* table, int count, ui
     const uint32_t tb = dt->group_base, te = tb + dt->n_groups;
     const uint32_t g1 = te < ge ? te : ge;  // this tensor's part of the run: [g0, g1)
     load_tables<kW>(dt, sm);
+    if (g0 == gb) wait_prerequisites();  // once, after the first table
     uint32_t g = g0 + warp;
     if (g < g1) {
       GroupIn in;
@@ -610,6 +640,8 @@ __device__ __forceinline__ void decode_split(const DevTensor* t, const SplitArgs
 __global__ void __launch_bounds__(kThreads, 1) decode_table_kernel(const DevTensor* __restrict__ ts,
                                                                     const __grid_constant__ SplitArgs a,
                                                                     int32_t* status) {
+  allow_dependents();
+  wait_prerequisites();  // the descriptor table itself was copied in by earlier stream work
   decode_split(ts, a, status);
 }
 
@@ -624,6 +656,7 @@ template <int N>
 __global__ void __launch_bounds__(kThreads, 1) decode_inline_kernel(const __grid_constant__ InlineBatch<N> b,
                                                                      const __grid_constant__ SplitArgs a,
                                                                      int32_t* status) {
+  allow_dependents();
   decode_split(b.t, a, status);
 }
 
@@ -796,19 +829,31 @@ int launch_parts(const DevTensor* h, const DevTensor* d_table, const Part part[2
     a.split = sp;
   }
   const int used = part[0].count + part[1].count;
+  // every launch allows programmatic dependent launch (see wait_prerequisites)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err;
   if (d_table) {
-    decode_table_kernel<<<grid, kThreads, sizeof(Smem), s>>>(d_table, a, status);
+    err = cudaLaunchKernelEx(&cfg, decode_table_kernel, d_table, a, status);
   } else if (used == 1) {
     InlineBatch<1> b;
     b.t[0] = h[0];
-    decode_inline_kernel<1><<<grid, kThreads, sizeof(Smem), s>>>(b, a, status);
+    err = cudaLaunchKernelEx(&cfg, decode_inline_kernel<1>, b, a, status);
   } else {
     if (used > kInlineMax) return ECF8_ERR_ARG;
     InlineBatch<kInlineMax> b;
     for (int i = 0; i < used; ++i) b.t[i] = h[i];
-    decode_inline_kernel<kInlineMax><<<grid, kThreads, sizeof(Smem), s>>>(b, a, status);
+    err = cudaLaunchKernelEx(&cfg, decode_inline_kernel<kInlineMax>, b, a, status);
   }
-  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
+  if (err != cudaSuccess || cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   g_launches.fetch_add(1);
   return ECF8_OK;
 }
