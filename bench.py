@@ -558,6 +558,49 @@ def run_pipeline(args):
             f.write(json.dumps(line) + "\n")
 
 
+def run_encode(args):
+    """Encoder throughput on the Llama-3-8B layer: the GPU encoder (histogram
+    kernel, host codebook, encode kernels) against the library's multithreaded
+    host encoder, every GPU blob checked byte for byte against the host one."""
+    import torch
+    L = load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    specs = synth.llama3_8b_layer().tensors
+    xs = [t.generate() for t in specs]
+    d_xs = [torch.from_numpy(x).to(dev) for x in xs]
+    n = sum(x.size for x in xs)
+    host_blobs = []
+    t0 = time.perf_counter()
+    for x in xs:
+        host_blobs.append(L.encode(x))
+    host_s = time.perf_counter() - t0
+    for x, d, hb in zip(xs, d_xs, host_blobs):
+        assert np.array_equal(L.encode_device(d).cpu().numpy(), hb)
+    reps = max(1, args.steps // 20)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        for d in d_xs:
+            L.encode_device(d)
+    e1.record()
+    torch.cuda.synchronize()
+    wall = (time.perf_counter() - t0) / reps
+    dev_ms = e0.elapsed_time(e1) / reps
+    line = {"workload": "encode_llama3_8b_layer_sas1.8", "n_bytes": n,
+            "gpu_encode_gbps_fp8_in": round(n / (dev_ms / 1e3) / 1e9, 2),
+            "gpu_encode_ms_per_layer": round(dev_ms, 4), "gpu_encode_wall_ms_per_layer": round(wall * 1e3, 3),
+            "host_encode_gbps_fp8_in": round(n / host_s / 1e9, 3), "host_cores": os.cpu_count(),
+            "note": "GPU time includes the histogram's device-to-host copy and the host codebook per tensor",
+            "blobs_equal_host_encoder": True}
+    print(json.dumps(line), flush=True)
+    if args.sweep_out:
+        with open(args.sweep_out, "a") as f:
+            f.write(json.dumps(line) + "\n")
+
+
 def load_library(build_only=False):
     from lossless_fp8_weight_b200 import _build
     _build.build()
@@ -580,6 +623,7 @@ def main():
     ap.add_argument("--moe-experts", type=int, default=256)
     ap.add_argument("--layers", type=int, default=80)
     ap.add_argument("--pipeline", action="store_true", help="decode-on-use pipeline beside FP8 GEMMs")
+    ap.add_argument("--encode", action="store_true", help="GPU encoder against the host encoder")
     ap.add_argument("--pipeline-layers", type=int, default=8)
     ap.add_argument("--pipeline-tokens", type=int, default=2048)
     ap.add_argument("--pipeline-ctas", type=lambda v: [int(c) for c in v.split(",")], default=[148, 74, 37, 18])
@@ -593,6 +637,8 @@ def main():
         return run_sweep(args)
     if args.pipeline:
         return run_pipeline(args)
+    if args.encode:
+        return run_encode(args)
 
     import torch
     import torch.distributed as dist

@@ -188,6 +188,35 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
  *    nothing.  Other arguments and errors are as for ecf8_decode_batched. */
 int ecf8_decode_batched_noalloc(const ecf8_tensor* tensors, int count, int32_t* d_status, cudaStream_t s);
 
+/* ---------------------------------------------------------------------------
+ * Encoding on the GPU (the same blob as ecf8_encode, byte for byte).  The
+ * histogram and every per-weight step run in kernels; the 16-symbol code and
+ * the header/decode-table prefix are built on the host.
+ *   ecf8_histogram_device(d_x, n, d_hist, s);          -- device counts
+ *   copy d_hist to the host, ecf8_build_codebook(hist, 16, &cb);
+ *   ecf8_encoded_size(hist, n, &cb, C, T, &bytes);      -- blob size
+ *   ecf8_encode_device(d_x, n, hist, &cb, C, T, d_blob, bytes, &bytes, ws, ws_bytes, s);
+ * d_fp8, d_hist, d_blob and the workspace are device memory, 16-byte aligned.
+ */
+
+/* Exponent histogram of n E4M3 bytes in device memory into d_hist[16]
+ * (device, uint64; zeroed by the call).  Asynchronous on stream s. */
+int ecf8_histogram_device(const uint8_t* d_fp8, size_t n, uint64_t* d_hist, cudaStream_t s);
+
+/* Bytes of device workspace ecf8_encode_device needs for n weights. */
+size_t ecf8_encode_device_workspace_size(size_t n);
+
+/* Encode n E4M3 bytes in device memory into d_blob (device, blob_cap bytes):
+ * the blob ecf8_encode writes for the same input, codebook and layout.
+ * hist (host) is the input's exponent histogram, which fixes the blob's size;
+ * cb must give every exponent that occurs a code (ECF8_ERR_CODEBOOK
+ * otherwise).  Asynchronous on stream s; *blob_bytes is set on return.
+ * Errors: ECF8_ERR_ARG, ECF8_ERR_ALIGN, ECF8_ERR_CODEBOOK, ECF8_ERR_CAPACITY,
+ * ECF8_ERR_WORKSPACE, ECF8_ERR_CUDA. */
+int ecf8_encode_device(const uint8_t* d_fp8, size_t n, const uint64_t hist[16], const ecf8_codebook* cb,
+                       uint32_t chunk_bytes, uint32_t group_chunks, void* d_blob, size_t blob_cap,
+                       size_t* blob_bytes, void* d_workspace, size_t workspace_bytes, cudaStream_t s);
+
 /* ecf8_decode_batched with the persistent grid capped at max_ctas CTAs (one
  * CTA occupies a whole SM's shared memory), so that a decode running beside
  * other kernels leaves them the remaining SMs.  max_ctas = 0: one CTA per SM.

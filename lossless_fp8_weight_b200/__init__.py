@@ -92,6 +92,11 @@ _lib.ecf8_batched_workspace_size.restype = _sz
 _lib.ecf8_decode_batched.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p]
 _lib.ecf8_decode_batched_noalloc.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _p]
 _lib.ecf8_decode_batched_ctas.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p, _u32]
+_lib.ecf8_histogram_device.argtypes = [_p, _sz, _p, _p]
+_lib.ecf8_encode_device_workspace_size.argtypes = [_sz]
+_lib.ecf8_encode_device_workspace_size.restype = _sz
+_lib.ecf8_encode_device.argtypes = [_p, _sz, _p, ctypes.POINTER(Codebook), _u32, _u32, _p, _sz, ctypes.POINTER(_sz),
+                                    _p, _sz, _p]
 
 
 class LayerTensor(ctypes.Structure):
@@ -170,6 +175,40 @@ def encode(fp8, codebook: Optional[Codebook] = None, chunk_bytes: int = DEFAULT_
     _check(_lib.ecf8_encode(x.ctypes.data, x.size, ctypes.byref(cb), chunk_bytes, group_chunks, blob.ctypes.data,
                             blob.size, ctypes.byref(got)), "ecf8_encode")
     assert got.value == blob.size
+    return blob
+
+
+def histogram_device(d_fp8, stream=None) -> np.ndarray:
+    """Exponent histogram of a CUDA uint8 tensor, computed on the GPU (the
+    call waits for it and returns a host array)."""
+    import torch
+    n = d_fp8.numel()
+    d_hist = torch.empty(16, dtype=torch.int64, device=d_fp8.device)
+    _check(_lib.ecf8_histogram_device(_ptr(d_fp8), n, _ptr(d_hist), _stream(stream)), "ecf8_histogram_device")
+    return d_hist.cpu().numpy().astype(np.uint64)
+
+
+def encode_device(d_fp8, codebook: Optional[Codebook] = None, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
+                  group_chunks: int = DEFAULT_GROUP_CHUNKS, max_len: int = 16, stream=None, hist=None):
+    """Compress a CUDA uint8 tensor of E4M3 bytes on the GPU; returns the blob
+    as a CUDA uint8 tensor (the same bytes as ``encode`` of the same input)."""
+    import torch
+    x = d_fp8.reshape(-1)
+    if x.dtype != torch.uint8:
+        x = x.view(torch.uint8)
+    n = x.numel()
+    h = histogram_device(x, stream) if hist is None else np.ascontiguousarray(np.asarray(hist, dtype=np.uint64))
+    cb = codebook if codebook is not None else build_codebook(h, max_len)
+    size = ctypes.c_size_t(0)
+    _check(_lib.ecf8_encoded_size(h.ctypes.data, n, ctypes.byref(cb), chunk_bytes, group_chunks, ctypes.byref(size)),
+           "ecf8_encoded_size")
+    blob = torch.empty(size.value, dtype=torch.uint8, device=x.device)
+    ws = torch.empty(max(16, _lib.ecf8_encode_device_workspace_size(n)), dtype=torch.uint8, device=x.device)
+    got = ctypes.c_size_t(0)
+    _check(_lib.ecf8_encode_device(_ptr(x), n, h.ctypes.data, ctypes.byref(cb), chunk_bytes, group_chunks, _ptr(blob),
+                                   blob.numel(), ctypes.byref(got), _ptr(ws), ws.numel(), _stream(stream)),
+           "ecf8_encode_device")
+    assert got.value == blob.numel()
     return blob
 
 

@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libecf8.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("ecf8_host.cpp", "ecf8_decode.cu", "ecf8_pipeline.cpp")]
+SOURCES = [os.path.join(CSRC, f) for f in ("ecf8_host.cpp", "ecf8_decode.cu", "ecf8_pipeline.cpp", "ecf8_encode.cu")]
 HEADERS = [os.path.join(ROOT, "include", "ecf8.h"), os.path.join(CSRC, "ecf8_format.h")]
 
 NVCC_FLAGS = [

@@ -55,6 +55,13 @@ inline bool compute_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t 
   return true;
 }
 
+// Host side of the device encoder (ecf8_host.cpp): checks the codebook
+// against the tensor's histogram and lays the blob out; writes the header and
+// decode-table section, bytes [0, gaps_off), the same as ecf8_encode does.
+int prepare_blob(const ecf8_codebook* cb, const uint64_t hist[16], uint64_t n, uint32_t chunk_bytes,
+                 uint32_t group_chunks, Layout* L, uint16_t code[16]);
+void write_blob_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t code[16]);
+
 // What a decode kernel needs to know about one tensor, with device pointers
 // already resolved into the blob's sections.
 struct alignas(16) DevTensor {

@@ -239,6 +239,35 @@ void pack_range(const uint8_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t 
   for (; boundary < bit1 && chunk < chunks; boundary += chunk_bits, ++chunk) put_gap(chunk, bit1 - boundary, i1);
 }
 
+// The header and the decode-table section of a blob; bytes [0, gaps_off)
+// must already be zero.
+void write_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t* code, uint8_t max_len,
+                  uint32_t chunk_bytes, uint32_t group_chunks) {
+  const uint64_t n = L.n;
+  store_le32(blob + 0, kMagic);
+  store_le32(blob + 4, kVersion);
+  store_le64(blob + 8, n);
+  store_le64(blob + 16, L.code_bits);
+  store_le32(blob + 24, chunk_bytes);
+  store_le32(blob + 28, group_chunks);
+  store_le32(blob + 32, (uint32_t)L.groups);
+  store_le32(blob + 36, kLutBits);
+  store_le32(blob + 40, n ? max_len : 0);
+  store_le32(blob + 44, kHeaderBytes);
+  store_le64(blob + 48, L.lut_off);
+  store_le64(blob + 56, L.gaps_off);
+  store_le64(blob + 64, L.groups_off);
+  store_le64(blob + 72, L.stream_off);
+  store_le64(blob + 80, L.nib_off);
+  store_le64(blob + 88, L.total);
+  memcpy(blob + 96, cb->len, 16);
+  if (n) {
+    std::vector<uint32_t> table(kLutEntries);
+    build_table(cb->len, code, table.data());
+    memcpy(blob + L.lut_off, table.data(), 4 * kLutEntries);
+  }
+}
+
 bool codebook_ok(const ecf8_codebook* cb, uint16_t* code_out) {
   uint16_t code[16];
   if (!canonical(cb->len, code)) return false;
@@ -341,30 +370,7 @@ int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t 
 
   // zero everything but the nibble section, which is written whole below
   memset(blob, 0, L.nib_off);
-
-  store_le32(blob + 0, kMagic);
-  store_le32(blob + 4, kVersion);
-  store_le64(blob + 8, n);
-  store_le64(blob + 16, L.code_bits);
-  store_le32(blob + 24, chunk_bytes);
-  store_le32(blob + 28, group_chunks);
-  store_le32(blob + 32, (uint32_t)L.groups);
-  store_le32(blob + 36, kLutBits);
-  store_le32(blob + 40, n ? max_len : 0);
-  store_le32(blob + 44, kHeaderBytes);
-  store_le64(blob + 48, L.lut_off);
-  store_le64(blob + 56, L.gaps_off);
-  store_le64(blob + 64, L.groups_off);
-  store_le64(blob + 72, L.stream_off);
-  store_le64(blob + 80, L.nib_off);
-  store_le64(blob + 88, L.total);
-  memcpy(blob + 96, cb->len, 16);
-
-  if (n) {
-    std::vector<uint32_t> table(kLutEntries);
-    build_table(cb->len, code, table.data());
-    memcpy(blob + L.lut_off, table.data(), 4 * kLutEntries);
-  }
+  write_prefix(blob, L, cb, code, max_len, chunk_bytes, group_chunks);
 
   uint32_t* stream = reinterpret_cast<uint32_t*>(blob + L.stream_off);
   uint32_t* gaps = reinterpret_cast<uint32_t*>(blob + L.gaps_off);
@@ -453,3 +459,29 @@ int ecf8_blob_info(const void* blob_v, size_t size, ecf8_info* out) {
 }
 
 }  // extern "C"
+
+namespace ecf8 {
+
+int prepare_blob(const ecf8_codebook* cb, const uint64_t hist[16], uint64_t n, uint32_t chunk_bytes,
+                 uint32_t group_chunks, Layout* L, uint16_t code[16]) {
+  if (!cb || !hist || !L || !code) return ECF8_ERR_ARG;
+  if (!codebook_ok(cb, code)) return ECF8_ERR_CODEBOOK;
+  uint64_t bits = 0, total = 0;
+  for (int s = 0; s < 16; ++s) {
+    if (hist[s] && !cb->len[s]) return ECF8_ERR_CODEBOOK;
+    bits += hist[s] * cb->len[s];
+    total += hist[s];
+  }
+  if (total != n) return ECF8_ERR_ARG;
+  if (!compute_layout(n, bits, chunk_bytes, group_chunks, L)) return ECF8_ERR_ARG;
+  return ECF8_OK;
+}
+
+void write_blob_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t code[16]) {
+  memset(blob, 0, L.gaps_off);
+  uint8_t max_len = 0;
+  for (int s = 0; s < 16; ++s) max_len = std::max(max_len, cb->len[s]);
+  write_prefix(blob, L, cb, code, max_len, L.C, L.T);
+}
+
+}  // namespace ecf8
