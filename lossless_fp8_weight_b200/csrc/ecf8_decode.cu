@@ -547,6 +547,12 @@ __device__ __forceinline__ int find_tensor(const DevTensor* ts, int count, uint3
   return lo;
 }
 
+// A CTA that enters a new tensor part way through its run rebuilds its table
+// and first waits for all its warps to finish the previous tensor: each
+// tensor's cost range starts with this much (about 18 groups' worth), so such
+// CTAs take fewer groups.
+constexpr uint64_t kTensorSetupCost = 100000;
+
 // The group that starts at estimated cost c of the launch: in the tensor whose
 // cost range holds c, the first group whose cost range starts at or after c.
 // Non-decreasing in c, 0 at c = 0 and the launch's group count at its total
@@ -558,8 +564,8 @@ __device__ __forceinline__ uint32_t group_at_cost(const DevTensor* ts, int count
     if (ts[mid].cost_base <= c) lo = mid;
     else hi = mid - 1;
   }
-  const uint64_t w = ts[lo].group_cost;
-  uint64_t k = (c - ts[lo].cost_base + w - 1) / w;
+  const uint64_t w = ts[lo].group_cost, rel = c - ts[lo].cost_base;
+  uint64_t k = rel > kTensorSetupCost ? (rel - kTensorSetupCost + w - 1) / w : 0;
   if (k > ts[lo].n_groups) k = ts[lo].n_groups;
   return ts[lo].group_base + (uint32_t)k;
 }
@@ -723,17 +729,17 @@ int width_of(const ecf8_info* info) {
   return kNarrow;
 }
 
-// Estimated cost of decoding one group of a tensor, in units of one decoded
-// weight: a fixed part (fetch, scan, table walk over the group's 1 KB of
-// code stream), worth about 2560 weights on B200 with the wide table and
-// 1800 with the narrow one, plus the weights the group holds, which is 8192
-// bits over the mean code length.  Only the split of work between CTAs
-// depends on it, never the bytes decoded.
+// Estimated cost of decoding one group of a tensor, in units of about one
+// decoded weight, fitted to per-CTA timings on B200: with the narrow table a
+// group costs nearly the same whatever its code count (the walk over its 1 KB
+// of stream dominates), with the wide table the weights it holds (8192 bits
+// over the mean code length) add on top of the walk.  Only the split of work
+// between CTAs depends on it, never the bytes decoded.
 uint32_t group_cost(const ecf8_info* info) {
   const uint64_t bits = (uint64_t)kC * kT * 8;
   uint64_t codes = info->code_bits ? bits * info->n / info->code_bits : bits;
   if (codes > bits) codes = bits;
-  return (width_of(info) == kWide ? 2560u : 1800u) + (uint32_t)codes;
+  return width_of(info) == kWide ? 3250u + (uint32_t)codes : 5200u + (uint32_t)codes / 10u;
 }
 
 DevTensor make_dev(const ecf8_info* info, const void* d_blob, uint8_t* d_out) {
@@ -795,7 +801,7 @@ int build_table(const ecf8_tensor* tensors, int count, DevTensor* table, Part pa
     t.group_base = (uint32_t)part[k].groups;
     t.cost_base = part[k].cost;
     part[k].groups += t.n_groups;
-    part[k].cost += (uint64_t)t.n_groups * t.group_cost;
+    part[k].cost += kTensorSetupCost + (uint64_t)t.n_groups * t.group_cost;
     if (part[k].groups > 0xFFFFFFFFull) return ECF8_ERR_UNSUPPORTED;
     table[at[k]++] = t;
   }
@@ -823,10 +829,21 @@ int launch_parts(const DevTensor* h, const DevTensor* d_table, const Part part[2
   } else if (part[1].groups == 0) {
     a.split = grid;
   } else {
-    const double f = (double)part[0].cost / (double)(part[0].cost + part[1].cost);
-    uint32_t sp = (uint32_t)(f * grid + 0.5);
-    sp = sp < 1 ? 1 : sp > grid - 1 ? grid - 1 : sp;
-    a.split = sp;
+    // of the two whole CTA counts nearest the cost share, the one whose
+    // busier part finishes first
+    const double cw = (double)part[0].cost, cn = (double)part[1].cost;
+    const double f = cw / (cw + cn) * grid;
+    uint32_t best = 1;
+    double best_t = 0;
+    for (uint32_t sp : {(uint32_t)f, (uint32_t)f + 1}) {
+      sp = sp < 1 ? 1 : sp > grid - 1 ? grid - 1 : sp;
+      const double t = cw / sp > cn / (grid - sp) ? cw / sp : cn / (grid - sp);
+      if (best_t == 0 || t < best_t) {
+        best = sp;
+        best_t = t;
+      }
+    }
+    a.split = best;
   }
   const int used = part[0].count + part[1].count;
   // every launch allows programmatic dependent launch (see wait_prerequisites)
