@@ -16,18 +16,25 @@
 //  * decoding is a finite-state machine over bytes: a 4096-entry table in
 //    shared memory, indexed by (node of the code tree, next stream byte),
 //    gives every exponent whose code ends in that byte and the node after
-//    it.  Each lane first shifts its slice so that it starts at its first
-//    code (the gap), and zeroes the bits after its last code, so all lanes run
-//    the same fully unrolled 34-byte loop.  Zeros after a code boundary decode
-//    as repeats of the all-zero code, whose number is known and subtracted.
+//    it.  Entries are 64-bit when the code has a 1-bit length (up to 8 codes
+//    end in a byte) and 32-bit otherwise (at most 4), which halves the banks
+//    a warp's random lookups touch; the narrow walk also packs two bytes'
+//    exponents per step.  Each lane first shifts its slice so that it starts
+//    at its first code (the gap), and zeroes the bits after its last code, so
+//    all lanes run the same fully unrolled 34-byte loop.  Zeros after a code
+//    boundary decode as repeats of the all-zero code, whose number is known
+//    and subtracted.
 //  * exponents are parked 4 bits each in lane-private shared memory, then
-//    funnel-shifted into a 32-weight-aligned stage; 8 bytes of stage plus one
-//    8-byte nibble load become 16 output bytes (byte-permute + 3-input
-//    logic), and consecutive lanes store consecutive 16-byte vectors.
-//  * CTAs are persistent, one per SM, each over a contiguous run of groups;
-//    every warp fetches its next group's stream slice, gaps and offsets while
-//    it decodes the current one, and issues the current group's nibble loads
-//    before its walk.
+//    funnel-shifted into a 32-weight-aligned stage; 16 bytes of stage plus a
+//    16-byte nibble load become 32 output bytes (byte-permute + 3-input
+//    logic), and consecutive lanes store consecutive 32-byte vectors.
+//  * CTAs are persistent, one per SM.  A launch puts the wide-table tensors on
+//    CTAs [0, split) and the rest on the others; within each part every CTA
+//    takes a contiguous run of groups of equal estimated cost.  Every warp
+//    fetches its next group's stream slice, gaps and offsets while it decodes
+//    the current one, and issues the current group's nibble loads before its
+//    walk.  Launches allow programmatic dependent launch, so a decode builds
+//    its first table while the previous kernel on the stream drains.
 //
 // The path is HBM-bound integer work: no tensor cores.  Corrupt input is
 // reported through a status word; no access leaves its buffer and no loop
