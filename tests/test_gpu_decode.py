@@ -244,3 +244,28 @@ def test_batched_without_workspace_fails_loudly(env):
     with pytest.raises(L.Ecf8Error) as e:
         _batched(env, blobs, workspace=False)
     assert e.value.code == -8
+
+
+def test_back_to_back_decodes_into_one_buffer_keep_stream_order(env):
+    """Decodes launched back to back may start early (dependent launch) but
+    must not write before the previous grid ends: alternate two tensors into
+    one buffer with no synchronisation, reading a copy after each."""
+    L, torch = env
+    specs = [synth.alpha_sweep_point(1.7, 448.0).tensors[0], synth.alpha_sweep_point(1.5, 448.0).tensors[0]]
+    xs = [s.generate(begin=99, count=3_000_017) for s in specs]
+    infos, blobs = [], []
+    for x in xs:
+        b = L.encode(x)
+        infos.append(L.blob_info(b))
+        blobs.append(torch.from_numpy(b).cuda())
+    out = torch.empty(xs[0].size, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    copies = []
+    for k in range(12):
+        j = k % 2
+        L.decode(infos[j], blobs[j], out, status=status)
+        copies.append((j, out.clone()))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for j, c in copies:
+        assert np.array_equal(c.cpu().numpy(), xs[j])
