@@ -78,6 +78,7 @@ extern "C" {
 #define ECF8_STATUS_COUNT_MISMATCH 1 /* codes decoded in a group != its offset delta */
 #define ECF8_STATUS_BAD_CODE 2       /* bits that match no code */
 #define ECF8_STATUS_BAD_OFFSETS 4    /* group offsets not monotone or past n */
+#define ECF8_STATUS_BOUNDS 8         /* checked builds only: an index failed its bounds check */
 
 /* A canonical Huffman code over the 16 exponent values. */
 typedef struct ecf8_codebook {

@@ -8,6 +8,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libecf8.so")
+# the same library with every kernel store and table read bounds-checked
+# (-DECF8_CHECKED): a failed check sets ECF8_STATUS_BOUNDS instead of accessing
+CHECKED_SO = os.path.join(HERE, "libecf8_checked.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("ecf8_host.cpp", "ecf8_decode.cu", "ecf8_pipeline.cpp", "ecf8_encode.cu")]
 HEADERS = [os.path.join(ROOT, "include", "ecf8.h"), os.path.join(CSRC, "ecf8_format.h")]
 
@@ -27,22 +30,24 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(SO):
+def stale(so: str = SO) -> bool:
+    if not os.path.exists(so):
         return True
-    t = os.path.getmtime(SO)
+    t = os.path.getmtime(so)
     return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or stale():
-        cmd = [nvcc(), *NVCC_FLAGS, "-I" + os.path.join(ROOT, "include"), "-I" + CSRC, "-o", SO, *SOURCES, "-lgomp"]
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    so = CHECKED_SO if checked else SO
+    if force or stale(so):
+        cmd = [nvcc(), *NVCC_FLAGS, *(["-DECF8_CHECKED"] if checked else []), "-I" + os.path.join(ROOT, "include"),
+               "-I" + CSRC, "-o", so, *SOURCES, "-lgomp"]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.check_call(cmd)
-    return SO
+    return so
 
 
 if __name__ == "__main__":
     import sys
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, checked="--checked" in sys.argv))

@@ -102,6 +102,18 @@ static_assert(offsetof(Smem, warp) % 16 == 0, "warp areas must be 16-byte aligne
 static_assert(offsetof(Smem, fsm) % 16 == 0, "table must be aligned");
 static_assert(sizeof(Smem) <= 227 * 1024, "shared memory budget");
 
+// Checked builds (-DECF8_CHECKED, libecf8_checked.so) test each index a
+// store or a table read uses against its buffer; a failing one skips the
+// access and sets ECF8_STATUS_BOUNDS.  Release builds compile the tests away.
+#ifdef ECF8_CHECKED
+__device__ __forceinline__ bool in_bounds(bool ok, int32_t* status) {
+  if (!ok && status) atomicOr(status, ECF8_STATUS_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, int32_t*) { return true; }
+#endif
+
 // ---------------------------------------------------------------- decode tables
 
 // Canonical code and internal-node numbering, by one warp.  State 0 is the
@@ -344,7 +356,8 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   uint4 nv[kND];
 #pragma unroll
   for (int j = 0; j < kND; ++j)
-    if (lane + 32 * j < blocks) nv[j] = __ldg(nib + lane + 32 * j);
+    if (lane + 32 * j < blocks && in_bounds((off0 >> 5) + lane + 32 * j < (n + 31) / 32, status))
+      nv[j] = __ldg(nib + lane + 32 * j);
   const uint32_t* nib32 = reinterpret_cast<const uint32_t*>(nib);
   const uint32_t u0 = (uint32_t)(off0 & 31) >> 4;
   const uint32_t first_full = u0 + ((off0 & 15) ? 1u : 0u);
@@ -390,13 +403,13 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
 #pragma unroll
     for (int j = 0; j < kBytes; ++j) {
       const uint32_t idx = __byte_perm(sw[j >> 2], y, 0x7740u | (3u - (j & 3)));  // byte | node << 8
-      const uint2 e = sm->fsm[idx];
+      const uint2 e = in_bounds(idx < (uint32_t)(kStates * 256), status) ? sm->fsm[idx] : make_uint2(0, kError);
       y = e.y;
       acc |= e.x << sh;
       const uint32_t carry = __funnelshift_l(e.x, 0u, sh);
       sh += e.y >> 8;
       if (sh >= 32) {
-        priv[32 * words] = acc;
+        if (in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
         ++words;
         acc = carry;
         sh -= 32;
@@ -408,8 +421,10 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     const uint32_t* tab = reinterpret_cast<const uint32_t*>(sm->fsm);
 #pragma unroll
     for (int j = 0; j < kBytes; j += 2) {
-      const uint32_t e1 = tab[nidx(sw[j >> 2], y, 3u - (j & 3))];
-      const uint32_t e2 = tab[nidx(sw[(j + 1) >> 2], e1, 3u - ((j + 1) & 3))];
+      const uint32_t i1 = nidx(sw[j >> 2], y, 3u - (j & 3));
+      const uint32_t e1 = in_bounds(i1 < (uint32_t)(kStates * 256), status) ? tab[i1] : (uint32_t)kError << 16;
+      const uint32_t i2 = nidx(sw[(j + 1) >> 2], e1, 3u - ((j + 1) & 3));
+      const uint32_t e2 = in_bounds(i2 < (uint32_t)(kStates * 256), status) ? tab[i2] : (uint32_t)kError << 16;
       y = e2;
       const uint32_t n1 = e1 >> 24;
       const uint32_t p = (e1 & 0xFFFFu) | ((e2 & 0xFFFFu) << n1);
@@ -417,14 +432,14 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
       const uint32_t carry = __funnelshift_l(p, 0u, sh);
       sh += n1 + (e2 >> 24);
       if (sh >= 32) {
-        priv[32 * words] = acc;
+        if (in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
         ++words;
         acc = carry;
         sh -= 32;
       }
     }
   }
-  if (sh) priv[32 * words] = acc;
+  if (sh && in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
   const uint32_t emitted = 8 * words + sh / 4;
   const uint32_t extra = sm->tree.zero_codes[kPadBits - E];
   const uint32_t node = kW == kWide ? y & 0xFFu : (y >> 16) & 0xFFu;
@@ -436,7 +451,8 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   if (kW == kWide && blocks > 32u * kND) {
 #pragma unroll
     for (int j = 0; j < kND; ++j)
-      if (lane + 32 * (kND + j) < blocks) nv2[j] = __ldg(nib + lane + 32 * (kND + j));
+      if (lane + 32 * (kND + j) < blocks && in_bounds((off0 >> 5) + lane + 32 * (kND + j) < (n + 31) / 32, status))
+        nv2[j] = __ldg(nib + lane + 32 * (kND + j));
   }
 
   // K3: place -- warp-shuffle scan of the counts
@@ -467,8 +483,10 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   const uint32_t q = (uint32_t)(off0 & 31) + start;
   const uint32_t d0 = q >> 3, dl = cnt ? (q + cnt - 1) >> 3 : 0;
   if (cnt) {
-    stage[sidx<kW>(d0)] = 0;
-    stage[sidx<kW>(dl)] = 0;
+    if (in_bounds(sidx<kW>(dl) < (uint32_t)kStagePhys, status)) {
+      stage[sidx<kW>(d0)] = 0;
+      stage[sidx<kW>(dl)] = 0;
+    }
   }
   __syncwarp();
   if (cnt) {
@@ -478,17 +496,18 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     if (cnt & 7) priv[32 * (used - 1)] &= (1u << (4 * (cnt & 7))) - 1;
     const uint32_t nwd = dl - d0 + 1;  // destination words: used or used + 1
     uint32_t prev = priv[0];
-    atomicOr(&stage[sidx<kW>(d0)], prev << r);
+    if (in_bounds(sidx<kW>(d0) < (uint32_t)kStagePhys, status)) atomicOr(&stage[sidx<kW>(d0)], prev << r);
     uint32_t j = 1;
 #pragma unroll 4
     for (; j + 1 < nwd; ++j) {  // interior words belong to this lane alone
       const uint32_t cur = priv[32 * j];
-      stage[sidx<kW>(d0 + j)] = __funnelshift_l(prev, cur, r);
+      if (in_bounds(sidx<kW>(d0 + j) < (uint32_t)kStagePhys, status)) stage[sidx<kW>(d0 + j)] = __funnelshift_l(prev, cur, r);
       prev = cur;
     }
     if (nwd > 1) {
       const uint32_t cur = j < used ? priv[32 * j] : 0;
-      atomicOr(&stage[sidx<kW>(d0 + j)], __funnelshift_l(prev, cur, r));
+      if (in_bounds(sidx<kW>(d0 + j) < (uint32_t)kStagePhys, status))
+        atomicOr(&stage[sidx<kW>(d0 + j)], __funnelshift_l(prev, cur, r));
     }
   }
   __syncwarp();
@@ -504,17 +523,18 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   for (int j = 0; j < kND; ++j) {
     const uint32_t d = lane + 32 * j;
     if (2 * d + 2 <= end_full && (j > 0 || 2 * d >= first_full))  // first_full <= 2
-      put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv[j]);
+      if (in_bounds(base + 32ull * d + 32 <= n, status)) put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv[j]);
   }
   if (kW == kWide && end_full > 64u * kND) {
 #pragma unroll
     for (int j = 0; j < kND; ++j) {
       const uint32_t d = lane + 32 * (kND + j);
-      if (2 * d + 2 <= end_full) put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv2[j]);
+      if (2 * d + 2 <= end_full && in_bounds(base + 32ull * d + 32 <= n, status))
+        put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv2[j]);
     }
   }
   for (uint32_t d = lane + 32 * (kW == kWide ? 2 * kND : kND); 2 * d + 2 <= end_full; d += 32)
-    put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), __ldg(nib + d));
+    if (in_bounds(base + 32ull * d + 32 <= n, status)) put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), __ldg(nib + d));
   {
     // a whole unit whose block partner is not whole: unit first_full when it
     // is odd (lane 0), unit end_full - 1 when end_full is odd (lane 1)
@@ -527,7 +547,8 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
       uint32_t o[4];
       assemble8(ex.x, nb.x, o[0], o[1]);
       assemble8(ex.y, nb.y, o[2], o[3]);
-      *reinterpret_cast<uint4*>(out + base + 16ull * su) = make_uint4(o[0], o[1], o[2], o[3]);
+      if (in_bounds(base + 16ull * su + 16 <= n, status))
+        *reinterpret_cast<uint4*>(out + base + 16ull * su) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
   if (hr || tr) {
@@ -537,7 +558,7 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
       const uint32_t e = (stage[sidx<kW>(i >> 3)] >> (4 * (i & 7))) & 15u;
       const uint32_t k = lane & 7;
       const uint32_t v = (rw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
-      out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
+      if (in_bounds(p < n, status)) out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
     }
   }
   __syncwarp();  // the stage and private words are reused by this warp's next group
