@@ -601,6 +601,65 @@ def run_encode(args):
             f.write(json.dumps(line) + "\n")
 
 
+def run_bf16(args):
+    """BF16 variant: decode throughput on the Llama-3-8B decoder layer in BF16
+    (seven launches, one per projection, on one stream), every output checked
+    against its source weights first."""
+    import torch
+    L = load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    specs = synth.llama3_8b_layer_bf16().tensors
+    xs = [t.generate_bf16() for t in specs]
+    blobs = [L.bf16_encode(x) for x in xs]
+    infos = [L.bf16_blob_info(b) for b in blobs]
+    d_blobs = [torch.from_numpy(b).to(dev) for b in blobs]
+    d_tables = [torch.from_numpy(L.bf16_table(i)).to(dev) for i in infos]
+    d_outs = [torch.empty(i.n, dtype=torch.int16, device=dev) for i in infos]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one(k):
+        L.bf16_decode(infos[k], d_blobs[k], d_tables[k], d_outs[k], status, stream)
+
+    def layer():
+        for k in range(len(specs)):
+            one(k)
+
+    layer()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"decode status {int(status.item())}"
+    for x, d in zip(xs, d_outs):
+        if not np.array_equal(d.cpu().numpy().view(np.uint16), x):
+            raise SystemExit("BF16 decode mismatch in the benchmark configuration")
+    n = sum(int(i.n) for i in infos)
+    blob = sum(int(b.size) for b in blobs)
+    alg = blob + 2 * n + len(specs) * 32768
+    peak, peak_kind = measured_hbm_peak()
+    launches0 = L.launch_count()
+    ms = _time_launches(torch, layer, max(1, args.steps), args.warmup)
+    launches = (L.launch_count() - launches0) // (max(1, args.steps) + args.warmup)
+    per = []
+    for k, spec in enumerate(specs):
+        mk = _time_launches(torch, lambda: one(k), max(1, args.steps), args.warmup)
+        ak = int(blobs[k].size) + 2 * int(infos[k].n) + 32768
+        per.append({"tensor": spec.name, "n": int(infos[k].n), "ms": round(mk, 5),
+                    "gbps_bf16_out": round(2 * infos[k].n / mk / 1e6, 2),
+                    "roofline_frac": round(ak / mk / 1e6 / peak, 4)})
+    line = {"workload": "bf16_llama3_8b_layer_normal0.02", "dtype": "bf16 bits (u16)", "n_weights": n,
+            "compressed_bytes": blob, "ratio_vs_bf16": round(2 * n / blob, 4),
+            "bits_per_weight": round(8 * blob / n, 4), "ms_per_layer": round(ms, 5),
+            "gbps_bf16_out": round(2 * n / ms / 1e6, 2), "gpu_launches_per_layer": launches,
+            "roofline": {"bound": "hbm", "achieved": round(alg / ms / 1e6, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(alg / ms / 1e6 / peak, 4),
+                         "algorithmic_bytes": alg, "peak_source": f"{peak_kind} hbm_gbs"},
+            "l2": "inputs+outputs larger than L2 (no flush)", "per_tensor": per, "outputs_checked": True}
+    print(json.dumps(line), flush=True)
+    if args.sweep_out:
+        with open(args.sweep_out, "a") as f:
+            f.write(json.dumps(line) + "\n")
+
+
 def load_library(build_only=False):
     from lossless_fp8_weight_b200 import _build
     _build.build()
@@ -624,6 +683,7 @@ def main():
     ap.add_argument("--layers", type=int, default=80)
     ap.add_argument("--pipeline", action="store_true", help="decode-on-use pipeline beside FP8 GEMMs")
     ap.add_argument("--encode", action="store_true", help="GPU encoder against the host encoder")
+    ap.add_argument("--bf16", action="store_true", help="BF16 variant decode on the Llama-3-8B layer in BF16")
     ap.add_argument("--pipeline-layers", type=int, default=8)
     ap.add_argument("--pipeline-tokens", type=int, default=2048)
     ap.add_argument("--pipeline-ctas", type=lambda v: [int(c) for c in v.split(",")], default=[148, 74, 37, 18])
@@ -639,6 +699,8 @@ def main():
         return run_pipeline(args)
     if args.encode:
         return run_encode(args)
+    if args.bf16:
+        return run_bf16(args)
 
     import torch
     import torch.distributed as dist

@@ -51,6 +51,10 @@ def _load():
         lib.synth_e4m3.argtypes = [dbl]
         lib.synth_gaussian.restype = None
         lib.synth_gaussian.argtypes = [u64, u64, u64, dbl, p]
+        lib.synth_bf16.restype = ctypes.c_uint16
+        lib.synth_bf16.argtypes = [dbl]
+        lib.synth_gaussian_bf16.restype = None
+        lib.synth_gaussian_bf16.argtypes = [u64, u64, u64, dbl, p]
         lib.synth_sas_max_abs.restype = dbl
         lib.synth_sas_max_abs.argtypes = [u64, u64, dbl]
         lib.synth_sas.restype = None
@@ -75,6 +79,11 @@ def uniform(seed: int, counter: int) -> float:
 def e4m3(x: float) -> int:
     """RNE cast of one double to an E4M3FN byte, saturating at +-448."""
     return int(_load().synth_e4m3(float(x)))
+
+
+def bf16(x: float) -> int:
+    """BF16 bit pattern of one double (through float32, nearest even)."""
+    return int(_load().synth_bf16(float(x)))
 
 
 def normal_raw(seed: int, n: int, begin: int = 0) -> np.ndarray:
@@ -133,6 +142,16 @@ class TensorSpec:
             raise ValueError(self.dist)
         return out[:count]
 
+    def generate_bf16(self, begin: int = 0, count: Optional[int] = None) -> np.ndarray:
+        """Elements [begin, begin + count) as BF16 bit patterns (uint16):
+        sigma * N(0, 1) rounded to BF16 (normal tensors only)."""
+        if self.dist != "normal":
+            raise ValueError("BF16 tensors are drawn from the normal law")
+        count = self.n - begin if count is None else count
+        out = np.empty(count, dtype=np.uint16)
+        _load().synth_gaussian_bf16(self.seed, begin, count, self.sigma, out.ctypes.data)
+        return out
+
 
 @dataclass
 class Workload:
@@ -166,6 +185,14 @@ def llama3_8b_layer(alpha: float = 1.8, max_abs: float = 448.0) -> Workload:
     """Seven projections of one Llama-3-8B decoder layer, SaS alpha=1.8, max|w|=448."""
     return Workload("llama3_8b_layer_sas1.8", "Llama-3-8B decoder layer (7 tensors), SaS a=1.8, max|w|=448",
                     [TensorSpec(nm, r, c, _seed(2, i), "sas", alpha=alpha, max_abs=max_abs)
+                     for i, (nm, r, c) in enumerate(LLAMA3_8B_LAYER)])
+
+
+def llama3_8b_layer_bf16(sigma: float = 0.02) -> Workload:
+    """The seven Llama-3-8B decoder-layer projections in BF16, w ~ N(0, sigma^2)
+    (the BF16 variant's workload: a BF16 checkpoint layer)."""
+    return Workload("llama3_8b_layer_bf16_normal", f"Llama-3-8B decoder layer (7 tensors) BF16, w ~ N(0,1)*{sigma}",
+                    [TensorSpec(nm, r, c, _seed(6, i), "normal", sigma=sigma)
                      for i, (nm, r, c) in enumerate(LLAMA3_8B_LAYER)])
 
 

@@ -16,6 +16,7 @@
  * seed + (counter + 1) * golden_gamma.  Element i draws counters 2i and 2i+1.
  */
 #include <math.h>
+#include <string.h>
 #include <stdint.h>
 #include <stddef.h>
 
@@ -80,6 +81,24 @@ void synth_gaussian(uint64_t seed, uint64_t begin, uint64_t count, double sigma,
   long long c = (long long)count;
 #pragma omp parallel for schedule(static)
   for (long long k = 0; k < c; ++k) out[k] = synth_e4m3(sigma * normal_at(seed, begin + (uint64_t)k));
+}
+
+/* BF16 bit pattern of a double: cast to float32 (round to nearest even),
+ * then keep the top 16 bits, rounding the dropped 16 to nearest even; NaN
+ * stays a quiet NaN.  BF16 is the upper half of an IEEE binary32. */
+uint16_t synth_bf16(double x) {
+  float f = (float)x;
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if (isnan(f)) return (uint16_t)((u >> 16) | 0x40);
+  return (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+/* out[i] = BF16(sigma * N_i), i in [begin, begin + count). */
+void synth_gaussian_bf16(uint64_t seed, uint64_t begin, uint64_t count, double sigma, uint16_t* out) {
+  long long c = (long long)count;
+#pragma omp parallel for schedule(static)
+  for (long long k = 0; k < c; ++k) out[k] = synth_bf16(sigma * normal_at(seed, begin + (uint64_t)k));
 }
 
 /* max |X_i| over i in [0, n) of the alpha-stable sample. */

@@ -289,6 +289,71 @@ uint64_t ecf8_launch_count(void);
 const char* ecf8_strerror(int code);
 int ecf8_abi_version(void);
 
+
+/* ---- BF16 variant (DFloat11 article §2-§3) --------------------------------
+ * A BF16 weight x splits into its 8-bit exponent field (x >> 7) & 0xFF, which
+ * is Huffman-coded per tensor over 256 values with codes of at most 16 bits,
+ * and one kept byte (sign << 7) | mantissa, stored verbatim.  The blob reuses
+ * the ECF8 stream, gap and group-offset layout; byte layout (little-endian):
+ *   0 magic "DF11" (0x31314644), 4 version 1, 8 n, 16 code_bits, 24 chunk
+ *   bytes, 28 group chunks, 32 groups, 36 max_len, 40 lens_off, 48 gaps_off,
+ *   56 groups_off, 64 stream_off, 72 kept_off, 80 total bytes; sections at
+ *   256-byte boundaries: 256 code lengths, 4-bit gaps (16-byte padded),
+ *   groups + 1 u64 offsets, stream (+16 zero bytes), n kept bytes (padded to
+ *   16). */
+typedef struct ecf8_bf16_info {
+  uint64_t n;
+  uint64_t code_bits;
+  uint64_t blob_bytes;
+  uint64_t lens_off, gaps_off, groups_off, stream_off, kept_off;
+  uint32_t chunk_bytes;
+  uint32_t group_chunks;
+  uint32_t n_groups;
+  uint32_t max_len;
+  uint8_t len[256];
+} ecf8_bf16_info;
+
+/* Code lengths (<= max_len, 1..16) for the exponents of n BF16 bit patterns:
+ * Huffman with (weight, id) ties, package-merge when deeper than max_len; a
+ * single present exponent gets a 1-bit code.  host in, host out. */
+int ecf8_bf16_code_lengths(const uint16_t* x, size_t n, uint32_t max_len, uint8_t len[256]);
+
+/* Exact blob size for x under len.  ECF8_ERR_CODEBOOK if an exponent of x has
+ * no code. */
+int ecf8_bf16_encoded_size(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,
+                           uint32_t group_chunks, size_t* bytes);
+
+/* Encode n BF16 bit patterns into blob (host, capacity cap); the bytes are
+ * those of the oracle's encoder for the same lengths.  ECF8_ERR_CAPACITY if
+ * cap is short; *bytes gets the size. */
+int ecf8_bf16_encode(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,
+                     uint32_t group_chunks, void* blob, size_t cap, size_t* bytes);
+
+/* Parse and validate a BF16 blob header (host memory, size bytes):
+ * ECF8_ERR_FORMAT on a bad magic, version or layout, ECF8_ERR_CODEBOOK on
+ * code lengths that are not a complete prefix code. */
+int ecf8_bf16_blob_info(const void* blob, size_t size, ecf8_bf16_info* out);
+
+/* Bytes of the decode table (32768): 256 tree nodes x 16 nibbles, 8 bytes an
+ * entry. */
+size_t ecf8_bf16_table_bytes(void);
+
+/* Fill h_table (host, ecf8_bf16_table_bytes() bytes) with the nibble-state
+ * table of info's code: entry (node, nibble) holds the exponents whose codes
+ * end inside the nibble (8 bits each, first lowest) and the next node with
+ * 8 x their count.  Copy it to the device once per codebook. */
+int ecf8_bf16_build_table(const ecf8_bf16_info* info, void* h_table);
+
+/* Decode one BF16 blob on the GPU.  d_blob (device, 16-byte aligned) holds
+ * info->blob_bytes; d_table (device, 16-byte aligned) the table of
+ * ecf8_bf16_build_table for the same info; d_out (device, 16-byte aligned)
+ * gets n uint16 BF16 bit patterns.  Requires chunk_bytes 32 and group_chunks
+ * 32 (ECF8_ERR_UNSUPPORTED otherwise).  Enqueued on stream; corrupt input
+ * ORs ECF8_STATUS_* bits into *d_status (may be null) and leaves the group's
+ * output unwritten. */
+int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, const void* d_table, uint16_t* d_out, size_t n,
+                     int32_t* d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -99,6 +99,31 @@ _lib.ecf8_encode_device.argtypes = [_p, _sz, _p, ctypes.POINTER(Codebook), _u32,
                                     _p, _sz, _p]
 
 
+class Bf16Info(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_uint64), ("code_bits", ctypes.c_uint64), ("blob_bytes", ctypes.c_uint64),
+                ("lens_off", ctypes.c_uint64), ("gaps_off", ctypes.c_uint64), ("groups_off", ctypes.c_uint64),
+                ("stream_off", ctypes.c_uint64), ("kept_off", ctypes.c_uint64),
+                ("chunk_bytes", ctypes.c_uint32), ("group_chunks", ctypes.c_uint32), ("n_groups", ctypes.c_uint32),
+                ("max_len", ctypes.c_uint32), ("len", ctypes.c_uint8 * 256)]
+
+    @property
+    def lengths(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.len), dtype=np.uint8).copy()
+
+    @property
+    def ratio(self) -> float:
+        return 2 * self.n / self.blob_bytes if self.blob_bytes else 0.0
+
+
+_lib.ecf8_bf16_code_lengths.argtypes = [_p, _sz, _u32, _p]
+_lib.ecf8_bf16_encoded_size.argtypes = [_p, _sz, _p, _u32, _u32, ctypes.POINTER(_sz)]
+_lib.ecf8_bf16_encode.argtypes = [_p, _sz, _p, _u32, _u32, _p, _sz, ctypes.POINTER(_sz)]
+_lib.ecf8_bf16_blob_info.argtypes = [_p, _sz, ctypes.POINTER(Bf16Info)]
+_lib.ecf8_bf16_table_bytes.restype = _sz
+_lib.ecf8_bf16_build_table.argtypes = [ctypes.POINTER(Bf16Info), _p]
+_lib.ecf8_bf16_decode.argtypes = [ctypes.POINTER(Bf16Info), _p, _p, _p, _sz, _p, _p]
+
+
 class LayerTensor(ctypes.Structure):
     _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("out_offset", ctypes.c_size_t)]
 
@@ -362,3 +387,63 @@ class Pipeline:
 
     def __del__(self):
         self.close()
+
+
+# ---- BF16 variant: 8-bit exponent field coded, sign + mantissa byte kept ----
+
+def _host_u16(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # a CPU torch tensor (bfloat16 or int16)
+        import torch
+        t = x.detach().contiguous().view(-1)
+        if t.dtype != torch.int16:
+            t = t.view(torch.int16)
+        x = t.numpy()
+    a = np.ascontiguousarray(np.asarray(x).reshape(-1))
+    if a.dtype != np.uint16:
+        a = a.view(np.uint16)
+    return a
+
+
+def bf16_code_lengths(x, max_len: int = 16) -> np.ndarray:
+    """Code lengths (256 entries) for the exponent fields of BF16 bit patterns."""
+    a = _host_u16(x)
+    ln = np.zeros(256, dtype=np.uint8)
+    _check(_lib.ecf8_bf16_code_lengths(a.ctypes.data, a.size, max_len, ln.ctypes.data), "ecf8_bf16_code_lengths")
+    return ln
+
+
+def bf16_encode(x, lengths=None, chunk_bytes: int = DEFAULT_CHUNK_BYTES, group_chunks: int = DEFAULT_GROUP_CHUNKS,
+                max_len: int = 16) -> np.ndarray:
+    """Compress BF16 weights (bit patterns as uint16, or a CPU bfloat16 tensor) into a blob."""
+    a = _host_u16(x)
+    ln = bf16_code_lengths(a, max_len) if lengths is None else np.ascontiguousarray(np.asarray(lengths, np.uint8))
+    size = ctypes.c_size_t(0)
+    _check(_lib.ecf8_bf16_encoded_size(a.ctypes.data, a.size, ln.ctypes.data, chunk_bytes, group_chunks,
+                                       ctypes.byref(size)), "ecf8_bf16_encoded_size")
+    blob = np.empty(size.value, dtype=np.uint8)
+    got = ctypes.c_size_t(0)
+    _check(_lib.ecf8_bf16_encode(a.ctypes.data, a.size, ln.ctypes.data, chunk_bytes, group_chunks, blob.ctypes.data,
+                                 blob.size, ctypes.byref(got)), "ecf8_bf16_encode")
+    assert got.value == blob.size
+    return blob
+
+
+def bf16_blob_info(blob) -> Bf16Info:
+    b = _host_u8(blob)
+    info = Bf16Info()
+    _check(_lib.ecf8_bf16_blob_info(b.ctypes.data, b.size, ctypes.byref(info)), "ecf8_bf16_blob_info")
+    return info
+
+
+def bf16_table(info: Bf16Info) -> np.ndarray:
+    """The decode table of info's code (host uint8 array; copy it to the device once)."""
+    t = np.zeros(int(_lib.ecf8_bf16_table_bytes()), dtype=np.uint8)
+    _check(_lib.ecf8_bf16_build_table(ctypes.byref(info), t.ctypes.data), "ecf8_bf16_build_table")
+    return t
+
+
+def bf16_decode(info: Bf16Info, d_blob, d_table, d_out, status=None, stream=None) -> None:
+    """Asynchronously decode one BF16 blob in device memory into d_out (n
+    uint16/bfloat16 elements) with the device copy of ``bf16_table(info)``."""
+    _check(_lib.ecf8_bf16_decode(ctypes.byref(info), _ptr(d_blob), _ptr(d_table), _ptr(d_out), info.n, _ptr(status),
+                                 _stream(stream)), "ecf8_bf16_decode")

@@ -11,7 +11,8 @@ SO = os.path.join(HERE, "libecf8.so")
 # the same library with every kernel store and table read bounds-checked
 # (-DECF8_CHECKED): a failed check sets ECF8_STATUS_BOUNDS instead of accessing
 CHECKED_SO = os.path.join(HERE, "libecf8_checked.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("ecf8_host.cpp", "ecf8_decode.cu", "ecf8_pipeline.cpp", "ecf8_encode.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("ecf8_host.cpp", "ecf8_decode.cu", "ecf8_pipeline.cpp", "ecf8_encode.cu",
+                                                 "ecf8_bf16_host.cpp", "ecf8_bf16_decode.cu")]
 HEADERS = [os.path.join(ROOT, "include", "ecf8.h"), os.path.join(CSRC, "ecf8_format.h")]
 
 NVCC_FLAGS = [

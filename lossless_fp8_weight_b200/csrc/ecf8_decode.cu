@@ -906,6 +906,10 @@ int launch_parts(const DevTensor* h, const DevTensor* d_table, const Part part[2
 }  // namespace
 }  // namespace ecf8
 
+namespace ecf8 {
+void note_launch() { g_launches.fetch_add(1); }
+}  // namespace ecf8
+
 using namespace ecf8;
 
 extern "C" {

@@ -62,6 +62,9 @@ int prepare_blob(const ecf8_codebook* cb, const uint64_t hist[16], uint64_t n, u
                  uint32_t group_chunks, Layout* L, uint16_t code[16]);
 void write_blob_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t code[16]);
 
+// Counts one kernel launch in ecf8_launch_count (ecf8_decode.cu).
+void note_launch();
+
 // What a decode kernel needs to know about one tensor, with device pointers
 // already resolved into the blob's sections.
 struct alignas(16) DevTensor {

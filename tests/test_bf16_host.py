@@ -1,0 +1,213 @@
+"""Host side of the BF16 variant (DFloat11 article §2-§3) in libecf8: the
+library encoder writes the oracle's bytes, the header parser agrees with the
+oracle's, the nibble-state decode table walks every stream back to its
+exponents, and an emulation of the GPU kernel's per-lane partition (gap, bit
+budget, zero-padding codes, warp scan, stage placement) reproduces the input
+(ECF8 walkthrough §3.2.1 for the gap / group-offset plan the kernel shares)."""
+import numpy as np
+import pytest
+
+import oracle
+import lossless_fp8_weight_b200 as L
+
+
+def _bf16_bits(f32) -> np.ndarray:
+    u = np.asarray(f32, dtype=np.float32).view(np.uint32)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _cases():
+    r = np.random.default_rng(11)
+    return {
+        "normal": _bf16_bits(r.standard_normal(40_003) * 0.02),
+        "random_bits": r.integers(0, 1 << 16, 30_001).astype(np.uint16),
+        "single_symbol": np.full(5000, 0x4049, dtype=np.uint16),
+        "two_symbols": np.where(r.random(7777) < 0.9, 0x3F80, 0x4000).astype(np.uint16),
+        "skewed_capped": (((np.minimum(r.geometric(0.5, 20_000), 200) + 20) << 7)
+                          | r.integers(0, 128, 20_000)).astype(np.uint16),
+        "one": np.array([0xBF80], dtype=np.uint16),
+        "empty": np.zeros(0, dtype=np.uint16),
+    }
+
+
+CASES = _cases()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("C,T", [(32, 32), (4, 1), (8, 3)])
+def test_library_encoder_writes_the_oracle_bytes(name, C, T):
+    x = CASES[name]
+    a = L.bf16_encode(x, chunk_bytes=C, group_chunks=T)
+    b = oracle.bf16_encode(x, chunk_bytes=C, group_chunks=T)
+    assert np.array_equal(a, b)
+    assert np.array_equal(L.bf16_code_lengths(x), oracle.bf16_blob_header(b)["lengths"])
+
+
+def test_given_lengths_and_a_length_cap():
+    x = CASES["skewed_capped"]
+    for cap in (9, 12, 16):
+        ln = L.bf16_code_lengths(x, cap)
+        assert ln.max() <= cap
+        assert np.array_equal(L.bf16_encode(x, lengths=ln), oracle.bf16_encode(x, lengths=ln))
+    # a non-optimal but complete code: every present exponent at length 8
+    ln = np.zeros(256, np.uint8)
+    ln[:] = 8
+    assert np.array_equal(L.bf16_encode(x, lengths=ln), oracle.bf16_encode(x, lengths=ln))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_blob_info_matches_the_header(name):
+    x = CASES[name]
+    blob = oracle.bf16_encode(x)
+    hd = oracle.bf16_blob_header(blob)
+    i = L.bf16_blob_info(blob)
+    assert i.n == x.size and i.code_bits == hd["code_bits"] and i.n_groups == hd["n_groups"]
+    assert i.max_len == hd["max_len"] and i.blob_bytes == blob.size
+    assert (i.stream_off, i.kept_off, i.gaps_off, i.groups_off) == (hd["stream_off"], hd["kept_off"],
+                                                                     hd["gaps_off"], hd["groups_off"])
+    assert np.array_equal(i.lengths, hd["lengths"])
+
+
+def test_blob_info_rejects_damaged_headers():
+    blob = oracle.bf16_encode(CASES["normal"])
+    for off, val in [(0, 0x00), (4, 2), (40, 7), (80, 1)]:
+        b = blob.copy()
+        b[off] ^= val if val else 0xFF
+        with pytest.raises(L.Ecf8Error):
+            L.bf16_blob_info(b)
+    b = blob.copy()
+    hd = oracle.bf16_blob_header(blob)
+    b[hd["lens_off"] + int(np.argmax(hd["lengths"]))] += 1  # breaks the Kraft sum
+    with pytest.raises(L.Ecf8Error):
+        L.bf16_blob_info(b)
+    with pytest.raises(L.Ecf8Error):
+        L.bf16_blob_info(blob[:100])
+
+
+def _table(info):
+    t = L.bf16_table(info).view(np.uint32).reshape(256 * 16, 2)
+    return t[:, 0].astype(np.uint64), t[:, 1].astype(np.uint64)
+
+
+def _stream_bits(blob, hd):
+    words = blob[hd["stream_off"]:hd["stream_off"] + 4 * ((hd["code_bits"] + 31) // 32)].view("<u4")
+    return np.unpackbits(words.astype(">u4").view(np.uint8))[:hd["code_bits"]]
+
+
+@pytest.mark.parametrize("name", [n for n in CASES if n != "empty"])
+def test_table_walk_decodes_the_whole_stream(name):
+    """Walk the table over the stream a nibble at a time from the root."""
+    x = CASES[name]
+    blob = oracle.bf16_encode(x)
+    hd = oracle.bf16_blob_header(blob)
+    syms, nxt = _table(L.bf16_blob_info(blob))
+    bits = _stream_bits(blob, hd)
+    bits = np.concatenate([bits, np.zeros((-bits.size) % 4, np.uint8)])
+    nibs = bits.reshape(-1, 4) @ np.array([8, 4, 2, 1])
+    node, out = 0, []
+    for v in nibs:
+        e = node * 16 + int(v)
+        k = int(nxt[e] >> 12) // 8
+        out += [(int(syms[e]) >> (8 * j)) & 0xFF for j in range(k)]
+        node = int(nxt[e] >> 4) & 0xFF
+        assert node != 255
+    lmin = int(hd["lengths"][hd["lengths"] > 0].min())
+    pad = (-hd["code_bits"]) % 4  # zero bits after the stream decode as the all-zeros code
+    extra = pad // lmin
+    assert len(out) == x.size + extra
+    assert np.array_equal(np.array(out[:x.size], dtype=np.uint16), (x >> 7) & 0xFF)
+
+
+def test_table_error_node_and_invalid_bits():
+    x = CASES["single_symbol"]
+    info = L.bf16_blob_info(oracle.bf16_encode(x))
+    syms, nxt = _table(info)
+    assert int(nxt[0 * 16 + 0] >> 12) == 32 and int(syms[0]) == 0x80808080  # four 0-bit codes of exponent 128
+    for v in range(1, 16):
+        assert (int(nxt[v]) >> 4) & 0xFF == 255  # a 1 bit is no code
+    assert all((int(nxt[255 * 16 + v]) >> 4) & 0xFF == 255 for v in range(16))  # the error node absorbs
+    # a single exponent with a 3-bit code: one exponent per three zero bits
+    ln = np.zeros(256, np.uint8)
+    ln[128] = 3
+    blob = oracle.bf16_encode(x, lengths=ln)
+    assert np.array_equal(oracle.bf16_decode(blob, x.size), x)
+    syms, nxt = _table(L.bf16_blob_info(blob))
+    node, got = 0, 0
+    for _ in range(6):  # 24 zero bits = 8 codes
+        e = node * 16
+        got += int(nxt[e] >> 12) // 8
+        node = int(nxt[e] >> 4) & 0xFF
+    assert got == 8 and node == 0
+
+
+def _emulate_kernel(blob, x_size):
+    """The GPU kernel's per-lane plan in numpy (C = T = 32): lane bits from its
+    gap to the next chunk's gap, 68-nibble walk over zero-padded bits, padding
+    codes removed by count, warp scan, byte placement relative to the group's
+    16-aligned base, then join with the kept bytes."""
+    hd = oracle.bf16_blob_header(blob)
+    info = L.bf16_blob_info(blob)
+    syms, nxt = _table(info)
+    lens = hd["lengths"]
+    lmin = int(lens[lens > 0].min())
+    gaps_b = blob[hd["gaps_off"]:hd["groups_off"]]
+    groups = blob[hd["groups_off"]:hd["groups_off"] + 8 * (hd["n_groups"] + 1)].view("<u8")
+    sbytes = blob[hd["stream_off"]:hd["kept_off"]]
+    kept = blob[hd["kept_off"]:hd["kept_off"] + x_size]
+    out = np.full(x_size, 0xDEAD, dtype=np.uint32)
+    nchunks = hd["n_groups"] * 32
+
+    def gap_of(c):
+        return (int(gaps_b[c // 2]) >> (4 * (c % 2))) & 15 if c < nchunks else 0
+
+    for g in range(hd["n_groups"]):
+        off0, off1 = int(groups[g]), int(groups[g + 1])
+        assert off1 - off0 <= 8192
+        counts, lane_syms = [], []
+        for lane in range(32):
+            c = g * 32 + lane
+            gap = gap_of(c)
+            gap_next = gap_of(c + 1) if (lane < 31 or g + 1 < hd["n_groups"]) else 0
+            bit0 = c * 256
+            left = max(hd["code_bits"] - bit0, 0)
+            stop = min(left, 256 + gap_next)
+            E = max(stop - gap, 0)
+            assert E <= 271
+            w = sbytes[32 * c:32 * c + 36]  # 9 words: the chunk and one more (inside the 16-byte tail)
+            assert w.size == 36
+            bits = np.unpackbits(w.view("<u4").astype(">u4").view(np.uint8))[gap:gap + 272].copy()
+            bits = np.concatenate([bits, np.zeros(272 - bits.size, np.uint8)])
+            bits[E:] = 0
+            node, got = 0, []
+            for j in range(68):
+                v = int(bits[4 * j:4 * j + 4] @ np.array([8, 4, 2, 1]))
+                e = node * 16 + v
+                k = int(nxt[e] >> 12) // 8
+                got += [(int(syms[e]) >> (8 * q)) & 0xFF for q in range(k)]
+                node = int(nxt[e] >> 4) & 0xFF
+            assert node != 255 and len(got) <= 4 * 69
+            extra = (272 - E) // lmin
+            assert len(got) >= extra
+            cnt = len(got) - extra
+            counts.append(cnt)
+            lane_syms.append(got[:cnt])
+        assert sum(counts) == off1 - off0
+        stage = np.zeros(8192 + 32, np.uint8)
+        start = 0
+        for lane in range(32):
+            q = (off0 & 15) + start
+            stage[q:q + counts[lane]] = lane_syms[lane]
+            start += counts[lane]
+        base = off0 & ~15
+        for p in range(off0, off1):
+            e = int(stage[p - base])
+            k = int(kept[p])
+            out[p] = ((k >> 7) << 15) | (e << 7) | (k & 0x7F)
+    return out.astype(np.uint16)
+
+
+@pytest.mark.parametrize("name", ["normal", "random_bits", "single_symbol", "two_symbols", "skewed_capped", "one"])
+def test_kernel_plan_emulation_reproduces_the_input(name):
+    x = CASES[name][:12_000]
+    blob = oracle.bf16_encode(x)
+    assert np.array_equal(_emulate_kernel(blob, x.size), x)
