@@ -619,12 +619,25 @@ def run_bf16(args):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def one(k):
-        L.bf16_decode(infos[k], d_blobs[k], d_tables[k], d_outs[k], status, stream)
+    def one(k, layout="auto"):  # on the current stream (the capture stream inside a graph)
+        L.bf16_decode(infos[k], d_blobs[k], d_tables[k], d_outs[k], status, layout=layout)
 
     def layer():
         for k in range(len(specs)):
             one(k)
+
+    def graphed(fn, reps):
+        """fn() reps times as one CUDA graph, so that host launch cost stays out of the timing."""
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+        stream.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        return g
 
     layer()
     torch.cuda.synchronize()
@@ -637,15 +650,32 @@ def run_bf16(args):
     alg = blob + 2 * n + len(specs) * 32768
     peak, peak_kind = measured_hbm_peak()
     launches0 = L.launch_count()
-    ms = _time_launches(torch, layer, max(1, args.steps), args.warmup)
-    launches = (L.launch_count() - launches0) // (max(1, args.steps) + args.warmup)
+    g_layer = graphed(layer, 1)
+    launches = L.launch_count() - launches0 - len(specs)  # the capture's launches (the warm call excluded)
+    ms = _time_launches(torch, g_layer.replay, max(1, args.steps), args.warmup)
     per = []
     for k, spec in enumerate(specs):
-        mk = _time_launches(torch, lambda: one(k), max(1, args.steps), args.warmup)
+        g_one = graphed(lambda: one(k), 10)
+        mk = _time_launches(torch, g_one.replay, max(1, args.steps), args.warmup) / 10
         ak = int(blobs[k].size) + 2 * int(infos[k].n) + 32768
         per.append({"tensor": spec.name, "n": int(infos[k].n), "ms": round(mk, 5),
                     "gbps_bf16_out": round(2 * infos[k].n / mk / 1e6, 2),
                     "roofline_frac": round(ak / mk / 1e6 / peak, 4)})
+    # one 58.7M-weight projection under every table layout that holds its code
+    big = max(range(len(specs)), key=lambda k: infos[k].n)
+    by_layout = {}
+    for layout in ("wide", "narrow", "narrow_lane", "byte"):
+        try:
+            one(big, layout)
+        except L.Ecf8Error:
+            continue
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert np.array_equal(d_outs[big].cpu().numpy().view(np.uint16), xs[big])
+        g_l = graphed(lambda: one(big, layout), 10)
+        ml = _time_launches(torch, g_l.replay, max(1, args.steps), args.warmup) / 10
+        al = int(blobs[big].size) + 2 * int(infos[big].n) + 32768
+        by_layout[layout] = {"ms": round(ml, 5), "roofline_frac": round(al / ml / 1e6 / peak, 4)}
     line = {"workload": "bf16_llama3_8b_layer_normal0.02", "dtype": "bf16 bits (u16)", "n_weights": n,
             "compressed_bytes": blob, "ratio_vs_bf16": round(2 * n / blob, 4),
             "bits_per_weight": round(8 * blob / n, 4), "ms_per_layer": round(ms, 5),
@@ -653,7 +683,11 @@ def run_bf16(args):
             "roofline": {"bound": "hbm", "achieved": round(alg / ms / 1e6, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(alg / ms / 1e6 / peak, 4),
                          "algorithmic_bytes": alg, "peak_source": f"{peak_kind} hbm_gbs"},
-            "l2": "inputs+outputs larger than L2 (no flush)", "per_tensor": per, "outputs_checked": True}
+            "timing": "CUDA graph of the layer's 7 launches, replayed; per tensor: graph of 10 launches "
+                      "(tensors whose blob + output fit in L2 run L2-warm there)",
+            "l2": "inputs+outputs larger than L2 (no flush)", "per_tensor": per,
+            "auto_layout": {spec.name: L.bf16_auto_layout(i) for spec, i in zip(specs, infos)},
+            f"{specs[big].name}_by_layout": by_layout, "outputs_checked": True}
     print(json.dumps(line), flush=True)
     if args.sweep_out:
         with open(args.sweep_out, "a") as f:

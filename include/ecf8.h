@@ -339,10 +339,17 @@ int ecf8_bf16_blob_info(const void* blob, size_t size, ecf8_bf16_info* out);
 size_t ecf8_bf16_table_bytes(void);
 
 /* Fill h_table (host, ecf8_bf16_table_bytes() bytes) with the nibble-state
- * table of info's code: entry (node, nibble) holds the exponents whose codes
- * end inside the nibble (8 bits each, first lowest) and the next node with
- * 8 x their count.  Copy it to the device once per codebook. */
+ * table of info's code: 256 nodes x 16 nibbles of two u32 words; entry
+ * (node, nibble) at index node * 16 + nibble holds the exponents whose codes
+ * end inside the nibble (8 bits each, first lowest) and (next node << 7) |
+ * (8 x their count) << 16.  Node 0 is the root; node ecf8_bf16_table_nodes()
+ * is the error node, which every invalid bit sequence reaches and never
+ * leaves.  Copy it to the device once per codebook. */
 int ecf8_bf16_build_table(const ecf8_bf16_info* info, void* h_table);
+
+/* Number of tree nodes of info's code (the decoder reads the table's first
+ * nodes + 1 nodes); 0 when the code lengths are not a valid code. */
+uint32_t ecf8_bf16_table_nodes(const ecf8_bf16_info* info);
 
 /* Decode one BF16 blob on the GPU.  d_blob (device, 16-byte aligned) holds
  * info->blob_bytes; d_table (device, 16-byte aligned) the table of
@@ -353,6 +360,26 @@ int ecf8_bf16_build_table(const ecf8_bf16_info* info, void* h_table);
  * output unwritten. */
 int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, const void* d_table, uint16_t* d_out, size_t n,
                      int32_t* d_status, cudaStream_t stream);
+
+/* Table layouts of the BF16 decoder.  WIDE: 64-bit (node, nibble) entries,
+ * any code.  NARROW: 32-bit (node, nibble) entries, codes of >= 2 bits.
+ * NARROW_LANE: NARROW copied once per lane (bank-conflict free), codes of
+ * >= 2 bits on at most 31 tree nodes.  BYTE: 64-bit (node, byte) entries,
+ * half the steps, codes of >= 2 bits on at most 31 tree nodes.  AUTO: WIDE
+ * when a 1-bit code exists, else BYTE when it holds, else NARROW. */
+#define ECF8_BF16_LAYOUT_AUTO (-1)
+#define ECF8_BF16_LAYOUT_WIDE 0
+#define ECF8_BF16_LAYOUT_NARROW 1
+#define ECF8_BF16_LAYOUT_NARROW_LANE 2
+#define ECF8_BF16_LAYOUT_BYTE 3
+
+/* The layout ecf8_bf16_decode picks for info's code (>= 0), or an error. */
+int ecf8_bf16_auto_layout(const ecf8_bf16_info* info);
+
+/* ecf8_bf16_decode with a given table layout; ECF8_ERR_UNSUPPORTED when the
+ * layout cannot hold info's code.  The output is the same for every layout. */
+int ecf8_bf16_decode_layout(const ecf8_bf16_info* info, const void* d_blob, const void* d_table, uint16_t* d_out,
+                            size_t n, int32_t* d_status, cudaStream_t stream, int layout);
 
 #ifdef __cplusplus
 }

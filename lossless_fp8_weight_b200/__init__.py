@@ -121,7 +121,12 @@ _lib.ecf8_bf16_encode.argtypes = [_p, _sz, _p, _u32, _u32, _p, _sz, ctypes.POINT
 _lib.ecf8_bf16_blob_info.argtypes = [_p, _sz, ctypes.POINTER(Bf16Info)]
 _lib.ecf8_bf16_table_bytes.restype = _sz
 _lib.ecf8_bf16_build_table.argtypes = [ctypes.POINTER(Bf16Info), _p]
+_lib.ecf8_bf16_table_nodes.argtypes = [ctypes.POINTER(Bf16Info)]
+_lib.ecf8_bf16_table_nodes.restype = _u32
 _lib.ecf8_bf16_decode.argtypes = [ctypes.POINTER(Bf16Info), _p, _p, _p, _sz, _p, _p]
+_lib.ecf8_bf16_decode_layout.argtypes = [ctypes.POINTER(Bf16Info), _p, _p, _p, _sz, _p, _p, _i32]
+_lib.ecf8_bf16_auto_layout.argtypes = [ctypes.POINTER(Bf16Info)]
+BF16_LAYOUTS = {"auto": -1, "wide": 0, "narrow": 1, "narrow_lane": 2, "byte": 3}
 
 
 class LayerTensor(ctypes.Structure):
@@ -442,8 +447,22 @@ def bf16_table(info: Bf16Info) -> np.ndarray:
     return t
 
 
-def bf16_decode(info: Bf16Info, d_blob, d_table, d_out, status=None, stream=None) -> None:
+def bf16_table_nodes(info: Bf16Info) -> int:
+    """Tree nodes of info's code; the node with this index is the table's error node."""
+    return int(_lib.ecf8_bf16_table_nodes(ctypes.byref(info)))
+
+
+def bf16_auto_layout(info: Bf16Info) -> str:
+    """The table layout ``bf16_decode`` picks for info's code."""
+    rc = _lib.ecf8_bf16_auto_layout(ctypes.byref(info))
+    if rc < 0:
+        raise Ecf8Error(rc, "ecf8_bf16_auto_layout")
+    return {v: k for k, v in BF16_LAYOUTS.items()}[rc]
+
+
+def bf16_decode(info: Bf16Info, d_blob, d_table, d_out, status=None, stream=None, layout: str = "auto") -> None:
     """Asynchronously decode one BF16 blob in device memory into d_out (n
-    uint16/bfloat16 elements) with the device copy of ``bf16_table(info)``."""
-    _check(_lib.ecf8_bf16_decode(ctypes.byref(info), _ptr(d_blob), _ptr(d_table), _ptr(d_out), info.n, _ptr(status),
-                                 _stream(stream)), "ecf8_bf16_decode")
+    uint16/bfloat16 elements) with the device copy of ``bf16_table(info)``;
+    ``layout`` forces one of the decoder's table layouts (same output)."""
+    _check(_lib.ecf8_bf16_decode_layout(ctypes.byref(info), _ptr(d_blob), _ptr(d_table), _ptr(d_out), info.n,
+                                        _ptr(status), _stream(stream), BF16_LAYOUTS[layout]), "ecf8_bf16_decode")

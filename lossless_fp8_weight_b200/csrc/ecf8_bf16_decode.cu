@@ -5,17 +5,39 @@
 // The same plan as the ECF8 decoder, with an 8-bit alphabet: one warp per
 // group of 32 chunks of 32 stream bytes; each lane shifts its slice to its
 // first code (the gap), zeroes the bits after its last code and walks 68
-// nibbles through a state machine (256 tree nodes x 16 nibbles, 64-bit
-// entries: the exponents that end in the nibble and the next node; the table
-// comes from the host, ecf8_bf16_build_table); zero-padding codes are
-// subtracted; a warp scan places each lane's exponents; they are packed a
-// byte each into lane-private shared memory, funnel-shifted into a byte stage,
-// and 16 exponents plus 16 kept bytes become 16 BF16 values per lane step.
+// nibbles through a state machine over the code tree (one entry per (node,
+// nibble): the exponents whose codes end inside the nibble, their count and
+// the next node); zero-padding codes are subtracted by count; a warp scan
+// places each lane's exponents; they are packed a byte each into lane-private
+// shared memory, funnel-shifted into a byte stage, and 16 exponents plus 16
+// kept bytes become 16 BF16 values per lane step.  The group's kept bytes are
+// loaded into registers before its walk, so that their DRAM latency overlaps
+// it; the next group's stream words are loaded before the current group is
+// processed.
+//
+// Three table layouts, chosen per tensor on the host:
+//  - wide: when a 1-bit code exists a nibble may end 4 codes; 64-bit entries
+//    {exponents, next node << 7 | 8 count << 16}, as the host builds them;
+//    a group may hold 8192 codes, so 13 warps fit an SM;
+//  - narrow: shortest code >= 2 bits, so a nibble ends at most 2 codes and an
+//    entry packs into 32 bits (exponents 0-15, node 16-23, 8 count 27-31); a
+//    group holds at most 4096 codes and a lane 128, which halves the warp's
+//    buffers, so 16 warps fit;
+//  - narrow, lane-private: as narrow, with trees of at most 31 nodes copied
+//    once per lane (entry i of lane l at word 32 i + l), so that each lane
+//    reads its own bank and a lookup is one shared-memory wavefront;
+//  - byte: shortest code >= 2 bits and at most 31 nodes: one entry per
+//    (node, byte), composed on the device from two nibble entries (a byte
+//    ends at most 4 codes: 64-bit entries {exponents, node << 11 | 8 count
+//    << 24}), so a lane walks 34 steps instead of 68 (the default for such
+//    codes: half the table steps, at the price of bank conflicts).
 // Corrupt input is reported through the status word; no access leaves its
 // buffer and no loop runs without a bound.
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "ecf8.h"
 #include "ecf8_format.h"
@@ -24,30 +46,30 @@ namespace ecf8_bf16 {
 namespace {
 
 constexpr int kC = 32, kT = 32;
-constexpr int kWords = kC / 4;               // stream words per chunk
-constexpr int kSpanBits = 8 * kC;            // 256
-constexpr int kNibbles = 68;                 // 272 bits: a lane may own up to 256 + 15 bits
+constexpr int kWords = kC / 4;             // stream words per chunk
+constexpr int kSpanBits = 8 * kC;          // 256
+constexpr int kNibbles = 68;               // 272 bits: a lane may own up to 256 + 15 bits
 constexpr int kPadBits = 4 * kNibbles;
-constexpr int kPrivWords = kNibbles + 1;     // <= 272 codes, 4 per word
-constexpr int kMaxCodes = kSpanBits * kT;    // 8192
-constexpr int kStageWords = kMaxCodes / 4 + 8;
-constexpr int kWarps = 8;
-constexpr int kThreads = 32 * kWarps;
-constexpr uint32_t kErr = 255;
+constexpr int kKeep = 8;                   // kept-byte units per lane loaded before the walk
 
+enum Layout { kWide = ECF8_BF16_LAYOUT_WIDE, kNarrow = ECF8_BF16_LAYOUT_NARROW,
+              kNarrowLane = ECF8_BF16_LAYOUT_NARROW_LANE, kByte = ECF8_BF16_LAYOUT_BYTE };
+
+template <int V>
+struct Cfg {
+  // codes a lane / a group can hold: shortest code 1 bit (wide) or >= 2 bits (the others)
+  static constexpr int kLaneCodes = V == kWide ? 4 * (kNibbles + 1) : 128;
+  static constexpr int kPrivWords = kLaneCodes / 4 + 1;
+  static constexpr int kMaxCodes = V == kWide ? kSpanBits * kT : kSpanBits * kT / 2;
+  static constexpr int kStageWords = (kMaxCodes + 32) / 4;  // 15 head bytes + codes, whole 16-byte units
+  static constexpr int kMaxWarps = V == kWide ? 13 : 16;
+};
+
+template <int V>
 struct alignas(16) WarpArea {
-  uint32_t priv[kPrivWords * 32];  // word k of lane l at k*32 + l
-  uint32_t stage[kStageWords];     // exponent byte i at byte i (from the group's 16-aligned base)
+  uint32_t priv[Cfg<V>::kPrivWords * 32];  // word k of lane l at k*32 + l
+  uint32_t stage[Cfg<V>::kStageWords];     // exponent byte i at byte i (from the group's 16-aligned base)
 };
-struct alignas(16) Smem {
-  uint2 table[256 * 16];  // (node << 4 | nibble) -> {exponents, next node << 4 | 8*count << 12}
-  uint16_t zero_codes[kPadBits + 1];
-  uint16_t pad_[7];
-  WarpArea warp[kWarps];
-};
-static_assert(offsetof(Smem, warp) % 16 == 0, "warp areas must be 16-byte aligned");
-static_assert(offsetof(WarpArea, stage) % 16 == 0, "stage must be 16-byte aligned");
-static_assert(sizeof(Smem) <= 227 * 1024, "shared memory budget");
 
 struct Args {
   const uint32_t* gaps;
@@ -57,6 +79,8 @@ struct Args {
   uint16_t* out;
   uint64_t n, code_bits;
   uint32_t n_groups, lmin;
+  uint32_t nodes;     // tree nodes; the error node is node `nodes`
+  uint32_t zc_off, warp_off;
 };
 
 struct GroupIn {
@@ -91,11 +115,112 @@ __device__ __forceinline__ uint32_t pair_bf16(uint32_t p, uint32_t q) {
   return p + q * 128u + (p & 0x00800080u) * 255u;
 }
 
-__device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, const Smem* sm, WarpArea* wa,
-                              int32_t* status) {
+// Unit u of the group: 16 weights from base + 16u, their exponents at stage
+// bytes 16u..16u+15.  Whole units take two 16-byte stores; the group's ragged
+// first and last unit store only the weights inside the group, whose
+// positions relative to base are [head, head + count).
+__device__ __forceinline__ void emit_unit(uint16_t* out_base, const uint4* st, uint32_t head, uint32_t count,
+                                          uint32_t u, uint4 kb) {
+  const uint4 ex = st[u];
+  const uint32_t e4[4] = {ex.x, ex.y, ex.z, ex.w}, k4[4] = {kb.x, kb.y, kb.z, kb.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    o[2 * w] = pair_bf16(__byte_perm(k4[w], 0u, 0x4140), __byte_perm(e4[w], 0u, 0x4140));
+    o[2 * w + 1] = pair_bf16(__byte_perm(k4[w], 0u, 0x4342), __byte_perm(e4[w], 0u, 0x4342));
+  }
+  const uint32_t r0 = 16 * u;
+  if (r0 >= head && r0 + 16 <= head + count) {
+    uint4* dst = reinterpret_cast<uint4*>(out_base + r0);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (r0 + k >= head && r0 + k < head + count) out_base[r0 + k] = (uint16_t)(o[k >> 1] >> (16 * (k & 1)));
+  }
+}
+
+__device__ __forceinline__ uint32_t nibble_of(const uint32_t* sw, int j) {
+  return (sw[j >> 3] >> (28 - 4 * (j & 7))) & 15u;
+}
+
+// One table step: the entry for the current node and the lane's next nibble
+// (or byte); gives the exponents (first lowest) and 8 x their count.
+template <int V>
+struct Walker {
+  // narrow entry: exponents bits 0-15, node bits 16-23, 8 x count bits 27-31
+  static constexpr int kSteps = kNibbles;
+  const uint8_t* table;
+  uint32_t lane_term;
+  uint32_t e = 0;
+  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t lane)
+      : table(t), lane_term(V == kNarrowLane ? lane * 4 : 0) {}
+  __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
+    const uint32_t nib = nibble_of(sw, j);
+    // lane-private: byte (node * 16 + nib) * 128 + lane * 4; shared: (node * 16 + nib) * 4
+    const uint32_t at = V == kNarrowLane ? (((e >> 5) & (0x1Fu << 11)) | (nib << 7) | lane_term)
+                                         : (((e >> 10) & (0xFFu << 6)) | (nib << 2));
+    e = *reinterpret_cast<const uint32_t*>(table + at);
+    syms = e & 0xFFFFu;
+    bits8 = e >> 27;
+  }
+  __device__ __forceinline__ uint32_t node() const { return (e >> 16) & 0xFFu; }
+};
+
+template <>
+struct Walker<kWide> {
+  static constexpr int kSteps = kNibbles;
+  const uint8_t* table;
+  uint32_t y = 0;
+  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t) : table(t) {}
+  __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
+    const uint2 e = *reinterpret_cast<const uint2*>(table + ((y & (0xFFu << 7)) | (nibble_of(sw, j) << 3)));
+    y = e.y;
+    syms = e.x;
+    bits8 = e.y >> 16;
+  }
+  __device__ __forceinline__ uint32_t node() const { return (y >> 7) & 0xFFu; }
+};
+
+template <>
+struct Walker<kByte> {
+  // entry (node, byte) at byte offset node * 2048 + byte * 8
+  static constexpr int kSteps = kNibbles / 2;
+  const uint8_t* table;
+  uint32_t y = 0;
+  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t) : table(t) {}
+  __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
+    const uint32_t byte = (sw[j >> 2] >> (24 - 8 * (j & 3))) & 0xFFu;
+    const uint2 e = *reinterpret_cast<const uint2*>(table + ((y & (0x1Fu << 11)) | (byte << 3)));
+    y = e.y;
+    syms = e.x;
+    bits8 = e.y >> 24;
+  }
+  __device__ __forceinline__ uint32_t node() const { return (y >> 11) & 0x1Fu; }
+};
+
+template <int V>
+__device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, const uint8_t* table,
+                              const uint16_t* zero_codes, WarpArea<V>* wa, int32_t* status) {
+  using C = Cfg<V>;
   const uint32_t lane = threadIdx.x & 31;
   const uint64_t off0 = in.off0, off1 = in.off1;
-  const bool offsets_ok = off0 <= off1 && off1 <= a.n && off1 - off0 <= (uint64_t)kMaxCodes;
+  const bool offsets_ok = off0 <= off1 && off1 <= a.n && off1 - off0 <= (uint64_t)C::kMaxCodes;
+
+  // the group's kept bytes, in flight during the walk
+  const uint64_t base = off0 & ~15ull;
+  const uint32_t head = (uint32_t)(off0 & 15);
+  const uint32_t count = offsets_ok ? (uint32_t)(off1 - off0) : 0u;
+  // no kept byte is read for a group whose offsets fail their check
+  const uint32_t units = offsets_ok ? (head + count + 15) >> 4 : 0u;
+  const uint4* kept_units = reinterpret_cast<const uint4*>(a.kept + base);
+  uint4 kp[kKeep];
+#pragma unroll
+  for (int i = 0; i < kKeep; ++i) {
+    const uint32_t u = lane + 32 * i;
+    kp[i] = u < units ? __ldg(kept_units + u) : make_uint4(0, 0, 0, 0);
+  }
 
   // the lane's bits run from its first code to the next lane's first code or the stream end
   const uint32_t gap = (in.gapw >> ((lane & 7) * 4)) & 15u;
@@ -115,28 +240,30 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
     sw[i] &= (uint32_t)(0xFFFFFFFF00000000ull >> keep);
   }
 
-  // the nibble machine: 68 steps, exponents packed a byte each
+  // the nibble machine: 68 steps, exponents packed a byte each (codes past
+  // the lane's capacity, which in a valid stream only the zero padding
+  // produces, are counted but not stored)
   uint32_t* priv = wa->priv + lane;
-  uint32_t y = 0, acc = 0, sh = 0, words = 0;
+  Walker<V> walk(table, lane);
+  uint32_t acc = 0, sh = 0, words = 0;
 #pragma unroll
-  for (int j = 0; j < kNibbles; ++j) {
-    const uint32_t nib = (sw[j >> 3] >> (28 - 4 * (j & 7))) & 15u;
-    const uint2 e = sm->table[(y & 0xFF0u) | nib];
-    y = e.y;
-    acc |= e.x << sh;
-    const uint32_t carry = __funnelshift_l(e.x, 0u, sh);
-    sh += e.y >> 12;
+  for (int j = 0; j < Walker<V>::kSteps; ++j) {
+    uint32_t syms, bits8;
+    walk.step(sw, j, syms, bits8);
+    acc |= syms << sh;
+    const uint32_t carry = __funnelshift_l(syms, 0u, sh);
+    sh += bits8;
     if (sh >= 32) {
-      if (words < (uint32_t)kPrivWords) priv[32 * words] = acc;
+      if (words < (uint32_t)C::kPrivWords) priv[32 * words] = acc;
       ++words;
       acc = carry;
       sh -= 32;
     }
   }
-  if (sh && words < (uint32_t)kPrivWords) priv[32 * words] = acc;
+  if (sh && words < (uint32_t)C::kPrivWords) priv[32 * words] = acc;
   const uint32_t emitted = 4 * words + sh / 8;
-  const uint32_t extra = sm->zero_codes[kPadBits - (E < (uint32_t)kPadBits ? E : (uint32_t)kPadBits)];
-  const bool bad = ((y >> 4) & 0xFFu) == kErr || emitted < extra || words > (uint32_t)kPrivWords;
+  const uint32_t extra = zero_codes[kPadBits - (E < (uint32_t)kPadBits ? E : (uint32_t)kPadBits)];
+  const bool bad = walk.node() == a.nodes || emitted < extra || emitted - extra > (uint32_t)C::kLaneCodes;
   const uint32_t cnt = bad ? 0 : emitted - extra;
 
   uint32_t incl = cnt;
@@ -159,9 +286,9 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
     return;
   }
 
-  // exponent bytes into the stage at byte (off0 mod 16) + start
+  // exponent bytes into the stage at byte head + start
   uint32_t* stage = wa->stage;
-  const uint32_t q = (uint32_t)(off0 & 15) + start;
+  const uint32_t q = head + start;
   const uint32_t d0 = q >> 2, dl = cnt ? (q + cnt - 1) >> 2 : 0;
   if (cnt) {
     stage[d0] = 0;
@@ -176,6 +303,7 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
     uint32_t prev = priv[0];
     atomicOr(&stage[d0], prev << r);
     uint32_t j = 1;
+#pragma unroll 4
     for (; j + 1 < nwd; ++j) {
       const uint32_t cur = priv[32 * j];
       stage[d0 + j] = __funnelshift_l(prev, cur, r);
@@ -189,83 +317,162 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
   __syncwarp();
 
   // 16 weights per lane step: 16 exponent bytes + 16 kept bytes -> 32 output bytes
-  const uint64_t base = off0 & ~15ull;
-  const uint32_t units = (uint32_t)(((off0 & 15) + (off1 - off0) + 15) >> 4);
-  const uint32_t first_full = (off0 & 15) ? 1u : 0u;
-  const uint32_t end_full = (units && (off1 & 15)) ? units - 1 : units;
   const uint4* st = reinterpret_cast<const uint4*>(stage);
-  for (uint32_t u = lane; u < end_full; u += 32) {
-    if (u < first_full) continue;
-    const uint4 ex = st[u];
-    const uint4 kb = __ldg(reinterpret_cast<const uint4*>(a.kept + base) + u);
-    const uint32_t e4[4] = {ex.x, ex.y, ex.z, ex.w}, k4[4] = {kb.x, kb.y, kb.z, kb.w};
-    uint32_t o[8];
+  uint16_t* out_base = a.out + base;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      o[2 * w] = pair_bf16(__byte_perm(k4[w], 0u, 0x4140), __byte_perm(e4[w], 0u, 0x4140));
-      o[2 * w + 1] = pair_bf16(__byte_perm(k4[w], 0u, 0x4342), __byte_perm(e4[w], 0u, 0x4342));
-    }
-    uint4* dst = reinterpret_cast<uint4*>(a.out + base + 16ull * u);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  for (int i = 0; i < kKeep; ++i) {
+    const uint32_t u = lane + 32 * i;
+    if (u < units) emit_unit(out_base, st, head, count, u, kp[i]);
   }
-  // the ragged first and last unit, one weight per lane (lanes 0-15 head, 16-31 tail)
-  const bool hr = units && first_full;
-  const bool tr = end_full < units && !(hr && end_full == 0);
-  const bool rg = lane < 16 ? hr : tr;
-  const uint32_t ru = lane < 16 ? 0u : end_full;
-  const uint64_t p = base + 16ull * ru + (lane & 15);
-  if (rg && p >= off0 && p < off1) {
-    const uint32_t i = 16 * ru + (lane & 15);
-    const uint32_t e = (stage[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-    const uint32_t k = a.kept[p];
-    a.out[p] = (uint16_t)(((k >> 7) << 15) | (e << 7) | (k & 0x7Fu));
-  }
+  for (uint32_t u = lane + 32 * kKeep; u < units; u += 32)
+    emit_unit(out_base, st, head, count, u, __ldg(kept_units + u));
   __syncwarp();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const uint2* __restrict__ d_table, Args a,
-                                                              int32_t* status) {
+// The host's 64-bit entry {exponents, next node << 7 | 8 count << 16} in the
+// narrow 32-bit form (the host picks a narrow layout only when no entry holds
+// more than two exponents).
+__device__ __forceinline__ uint32_t narrow_entry(uint2 w) {
+  return (w.x & 0xFFFFu) | (((w.y >> 7) & 0xFFu) << 16) | (((w.y >> 16) & 0x1Fu) << 27);
+}
+
+template <int V>
+__global__ void __launch_bounds__(Cfg<V>::kMaxWarps * 32, 1)
+    decode_kernel(const uint2* __restrict__ d_table, Args a, int32_t* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem* sm = reinterpret_cast<Smem*>(smem_raw);
-  const uint4* src = reinterpret_cast<const uint4*>(d_table);
-  uint4* dst = reinterpret_cast<uint4*>(sm->table);
-  // the walk masks every next-node field to 8 bits, so any table stays in range
-  for (int i = threadIdx.x; i < 256 * 16 / 2; i += kThreads) dst[i] = __ldg(src + i);
-  for (int z = threadIdx.x; z <= kPadBits; z += kThreads) sm->zero_codes[z] = (uint16_t)(z / a.lmin);
-  __syncthreads();
-  const uint32_t warp = threadIdx.x >> 5;
-  uint32_t g = blockIdx.x * kWarps + warp;
-  if (g >= a.n_groups) return;
+  const uint32_t warps = blockDim.x >> 5, warp = threadIdx.x >> 5;
+  uint32_t g = blockIdx.x * warps + warp;
   GroupIn in;
-  fetch_group(a, g, in);
-  for (; g < a.n_groups; g += gridDim.x * kWarps) {
+  if (g < a.n_groups) fetch_group(a, g, in);  // in flight while the table is staged
+
+  const uint32_t entries = (a.nodes + 1) * 16;
+  if (V == kWide) {
+    uint2* t = reinterpret_cast<uint2*>(smem_raw);
+#pragma unroll 8
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) t[i] = __ldg(d_table + i);
+  } else if (V == kNarrow) {
+    uint32_t* t = reinterpret_cast<uint32_t*>(smem_raw);
+#pragma unroll 8
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) t[i] = narrow_entry(__ldg(d_table + i));
+  } else if (V == kByte) {
+    // the nibble entries once into the first warp area, then two of them per (node, byte)
+    uint2* once = reinterpret_cast<uint2*>(smem_raw + a.warp_off);
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) once[i] = __ldg(d_table + i);
+    __syncthreads();
+    uint2* t = reinterpret_cast<uint2*>(smem_raw);
+    for (uint32_t i = threadIdx.x; i < (a.nodes + 1) * 256; i += blockDim.x) {
+      const uint32_t node = i >> 8, byte = i & 255;
+      const uint2 e1 = once[node * 16 + (byte >> 4)];
+      const uint32_t n1 = (e1.y >> 7) & 0xFFu, c1 = (e1.y >> 16) & 0x3Fu;
+      const uint2 e2 = once[(n1 <= a.nodes ? n1 : a.nodes) * 16 + (byte & 15)];
+      const uint32_t n2 = n1 == a.nodes ? a.nodes : (e2.y >> 7) & 0xFFu, c2 = (e2.y >> 16) & 0x3Fu;
+      t[i] = make_uint2(e1.x | (c1 < 32 ? e2.x << c1 : 0u), (n2 << 11) | ((c1 + c2) << 24));
+    }
+  } else {
+    // each entry read once into the first warp area, then copied to every lane's slot
+    uint32_t* once = reinterpret_cast<uint32_t*>(smem_raw + a.warp_off);
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) once[i] = narrow_entry(__ldg(d_table + i));
+    __syncthreads();
+    uint32_t* t = reinterpret_cast<uint32_t*>(smem_raw);
+    for (uint32_t i = threadIdx.x; i < entries * 32; i += blockDim.x) t[i] = once[i >> 5];
+  }
+  uint16_t* zero_codes = reinterpret_cast<uint16_t*>(smem_raw + a.zc_off);
+  for (int z = threadIdx.x; z <= kPadBits; z += blockDim.x) zero_codes[z] = (uint16_t)(z / a.lmin);
+  __syncthreads();
+  WarpArea<V>* wa = reinterpret_cast<WarpArea<V>*>(smem_raw + a.warp_off) + warp;
+  if (g >= a.n_groups) return;
+  for (; g < a.n_groups; g += gridDim.x * warps) {
     GroupIn nx;
-    const uint32_t gn = g + gridDim.x * kWarps;
+    const uint32_t gn = g + gridDim.x * warps;
     const bool more = gn < a.n_groups;
     if (more) fetch_group(a, gn, nx);
-    process_group(a, g, in, sm, &sm->warp[warp], status);
+    process_group<V>(a, g, in, smem_raw, zero_codes, wa, status);
     if (more) in = nx;
   }
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+uint32_t up16(uint32_t x) { return (x + 15) & ~15u; }
+
+template <int V>
+int launch(Args a, const void* d_table, int32_t* d_status, cudaStream_t s) {
+  const uint32_t entries = (a.nodes + 1) * 16;
+  const uint32_t table_bytes = V == kWide ? entries * 8 : V == kNarrow ? entries * 4
+                               : V == kNarrowLane ? entries * 128 : (a.nodes + 1) * 2048;
+  a.zc_off = table_bytes;
+  a.warp_off = up16(a.zc_off + 2 * (kPadBits + 1));
+  int dev = 0, sms = 0, smem_max = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
+      cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev))
+    return ECF8_ERR_CUDA;
+  if ((uint32_t)smem_max <= a.warp_off) return ECF8_ERR_UNSUPPORTED;
+  const uint32_t fit = ((uint32_t)smem_max - a.warp_off) / (uint32_t)sizeof(WarpArea<V>);
+  const uint32_t warps = fit < (uint32_t)Cfg<V>::kMaxWarps ? fit : (uint32_t)Cfg<V>::kMaxWarps;
+  if (warps == 0) return ECF8_ERR_UNSUPPORTED;
+  const uint32_t smem = a.warp_off + warps * (uint32_t)sizeof(WarpArea<V>);
+  if (cudaFuncSetAttribute(decode_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max))
+    return ECF8_ERR_CUDA;
+  const uint64_t ctas_needed = ((uint64_t)a.n_groups + warps - 1) / warps;
+  const uint32_t grid = (uint32_t)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
+  decode_kernel<V><<<grid, warps * 32, smem, s>>>(static_cast<const uint2*>(d_table), a, d_status);
+  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
+  ecf8::note_launch();
+  return ECF8_OK;
+}
 
 }  // namespace
 }  // namespace ecf8_bf16
 
 using namespace ecf8_bf16;
 
-extern "C" int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, const void* d_table, uint16_t* d_out,
-                                size_t n, int32_t* d_status, cudaStream_t s) {
-  if (!info || n != info->n) return ECF8_ERR_ARG;
-  if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
-  if (n == 0) return ECF8_OK;
-  if (!d_blob || !d_table || !d_out) return ECF8_ERR_ARG;
-  if (!aligned16(d_blob) || !aligned16(d_table) || !aligned16(d_out)) return ECF8_ERR_ALIGN;
+namespace ecf8_bf16 {
+namespace {
+
+uint32_t shortest(const ecf8_bf16_info* info) {
   uint32_t lmin = 16;
   for (int v = 0; v < 256; ++v)
     if (info->len[v] && info->len[v] < lmin) lmin = info->len[v];
+  return lmin;
+}
+
+bool layout_holds(int layout, uint32_t lmin, uint32_t nodes) {
+  switch (layout) {
+    case kWide: return true;
+    case kNarrow: return lmin >= 2;
+    case kNarrowLane:
+    case kByte: return lmin >= 2 && nodes + 1 <= 32;
+    default: return false;
+  }
+}
+
+}  // namespace
+}  // namespace ecf8_bf16
+
+extern "C" int ecf8_bf16_auto_layout(const ecf8_bf16_info* info) {
+  if (!info) return ECF8_ERR_ARG;
+  const uint32_t nodes = ecf8_bf16_table_nodes(info);
+  if (nodes == 0) return ECF8_ERR_CODEBOOK;
+  const uint32_t lmin = shortest(info);
+  if (lmin == 1) return kWide;
+  return nodes + 1 <= 32 ? kByte : kNarrow;
+}
+
+extern "C" int ecf8_bf16_decode_layout(const ecf8_bf16_info* info, const void* d_blob, const void* d_table,
+                                       uint16_t* d_out, size_t n, int32_t* d_status, cudaStream_t s, int layout) {
+  if (!info || n != info->n) return ECF8_ERR_ARG;
+  if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
+  if (n == 0) return ECF8_OK;
+  if (layout == ECF8_BF16_LAYOUT_AUTO) {
+    const int l = ecf8_bf16_auto_layout(info);
+    if (l < 0) return l;
+    layout = l;
+  }
+  if (!d_blob || !d_table || !d_out) return ECF8_ERR_ARG;
+  if (!aligned16(d_blob) || !aligned16(d_table) || !aligned16(d_out)) return ECF8_ERR_ALIGN;
+  const uint32_t nodes = ecf8_bf16_table_nodes(info);
+  if (nodes == 0) return ECF8_ERR_CODEBOOK;
+  const uint32_t lmin = shortest(info);
+  if (!layout_holds(layout, lmin, nodes)) return ECF8_ERR_UNSUPPORTED;
   const uint8_t* b = static_cast<const uint8_t*>(d_blob);
   Args a;
   a.gaps = reinterpret_cast<const uint32_t*>(b + info->gaps_off);
@@ -277,15 +484,17 @@ extern "C" int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, 
   a.code_bits = info->code_bits;
   a.n_groups = info->n_groups;
   a.lmin = lmin;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))
-    return ECF8_ERR_CUDA;
-  if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem)))
-    return ECF8_ERR_CUDA;
-  const uint64_t ctas_needed = ((uint64_t)a.n_groups + kWarps - 1) / kWarps;
-  const uint32_t grid = (uint32_t)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
-  decode_kernel<<<grid, kThreads, sizeof(Smem), s>>>(static_cast<const uint2*>(d_table), a, d_status);
-  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
-  ecf8::note_launch();
-  return ECF8_OK;
+  a.nodes = nodes;
+  a.zc_off = a.warp_off = 0;
+  switch (layout) {
+    case kWide: return launch<kWide>(a, d_table, d_status, s);
+    case kNarrow: return launch<kNarrow>(a, d_table, d_status, s);
+    case kNarrowLane: return launch<kNarrowLane>(a, d_table, d_status, s);
+    default: return launch<kByte>(a, d_table, d_status, s);
+  }
+}
+
+extern "C" int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, const void* d_table, uint16_t* d_out,
+                                size_t n, int32_t* d_status, cudaStream_t s) {
+  return ecf8_bf16_decode_layout(info, d_blob, d_table, d_out, n, d_status, s, ECF8_BF16_LAYOUT_AUTO);
 }

@@ -271,76 +271,101 @@ int ecf8_bf16_blob_info(const void* blob_v, size_t size, ecf8_bf16_info* out) {
 
 size_t ecf8_bf16_table_bytes(void) { return 256 * 16 * 8; }
 
-// Entry (node s, nibble v) at index s * 16 + v: x = the exponents whose codes
-// end inside the nibble, 8 bits each, first lowest; y = (next node << 4) |
-// (8 * count) << 12.  Node 0 is the root; the internal nodes at depth l are
-// the code values first[l] + count[l] + k (k < nint[l]) numbered from
-// ibase[l] (with a single exponent present, node d means d zero bits read);
-// node 255 is the error node, which absorbs everything.
-int ecf8_bf16_build_table(const ecf8_bf16_info* info, void* h_table) {
-  if (!info || !h_table) return ECF8_ERR_ARG;
-  const uint8_t* len = info->len;
+}  // extern "C"
+
+namespace {
+
+// The code tree as the table builder numbers it: node 0 is the root; the
+// internal nodes at depth l are the code values first[l] + count[l] + k
+// (k < nint[l]) numbered from ibase[l]; with a single exponent present, node
+// d means d zero bits read.  nodes = the number of nodes, also the index of
+// the error node.
+struct Tree {
   uint32_t count[kMaxLen + 1] = {0}, first[kMaxLen + 1] = {0}, base[kMaxLen + 1] = {0};
   uint32_t nint[kMaxLen + 1] = {0}, ibase[kMaxLen + 1] = {0};
   int max_len = 0, present = 0;
-  for (int s = 0; s < kSym; ++s)
-    if (len[s]) { ++count[len[s]]; ++present; max_len = std::max<int>(max_len, len[s]); }
   std::vector<int> sorted;
+  uint32_t nodes = 0;
+  bool ok = false;
+};
+
+Tree make_tree(const uint8_t* len) {
+  Tree t;
+  for (int s = 0; s < kSym; ++s)
+    if (len[s] && len[s] <= kMaxLen) { ++t.count[len[s]]; ++t.present; t.max_len = std::max<int>(t.max_len, len[s]); }
   for (int l = 1; l <= kMaxLen; ++l)
     for (int s = 0; s < kSym; ++s)
-      if (len[s] == l) sorted.push_back(s);
+      if (len[s] == l) t.sorted.push_back(s);
   uint32_t c = 0, b = 0;
   for (int l = 1; l <= kMaxLen; ++l) {
-    c = (c + count[l - 1]) << 1;
-    first[l] = c;
-    base[l] = b;
-    b += count[l];
+    c = (c + t.count[l - 1]) << 1;
+    t.first[l] = c;
+    t.base[l] = b;
+    b += t.count[l];
   }
-  nint[0] = 1;
+  t.nint[0] = 1;
   uint32_t states = 1;
-  bool ok = present >= 1;
+  t.ok = t.present >= 1;
   for (int l = 1; l <= kMaxLen; ++l) {
-    long long k = l < max_len ? 2ll * nint[l - 1] - count[l] : 0;
-    if (k < 0) { ok = false; k = 0; }
-    nint[l] = (uint32_t)k;
-    ibase[l] = states;
+    long long k = l < t.max_len ? 2ll * t.nint[l - 1] - t.count[l] : 0;
+    if (k < 0) { t.ok = false; k = 0; }
+    t.nint[l] = (uint32_t)k;
+    t.ibase[l] = states;
     states += (uint32_t)k;
   }
-  if (present == 1) states = (uint32_t)max_len;  // node d = d zero bits read
-  if (states > 255) ok = false;
-  const uint32_t kErr = 255;
-  // node -> (depth, value)
+  if (t.present == 1) states = (uint32_t)t.max_len;
+  if (states > 255) t.ok = false;
+  t.nodes = t.ok ? states : 0;
+  return t;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint32_t ecf8_bf16_table_nodes(const ecf8_bf16_info* info) { return info ? make_tree(info->len).nodes : 0; }
+
+// Entry (node s, nibble v) at index s * 16 + v: x = the exponents whose codes
+// end inside the nibble, 8 bits each, first lowest; y = (next node << 7) |
+// (8 * count) << 16, i.e. the next node's byte offset in the table and the
+// bits the exponents take when packed a byte each.  Every entry of the
+// error node (index = nodes) and of the unused nodes above it leads to the
+// error node.
+int ecf8_bf16_build_table(const ecf8_bf16_info* info, void* h_table) {
+  if (!info || !h_table) return ECF8_ERR_ARG;
+  const Tree T = make_tree(info->len);
+  const uint32_t err = T.nodes;
   auto step = [&](uint32_t s, uint32_t bit, int* sym) -> uint32_t {
     *sym = -1;
-    if (!ok || s >= states) return kErr;
-    if (present == 1) {  // one symbol, code max_len zero bits: a 1 bit is no code
-      if (bit) return kErr;
-      if ((int)s + 1 < max_len) return s + 1;
-      *sym = sorted[0];
+    if (!T.ok || s >= T.nodes) return err;
+    if (T.present == 1) {  // one exponent, code max_len zero bits: a 1 bit is no code
+      if (bit) return err;
+      if ((int)s + 1 < T.max_len) return s + 1;
+      *sym = T.sorted[0];
       return 0;
     }
     uint32_t l = 0, v = 0;
-    for (int d = 1; d < max_len; ++d)
-      if (s >= ibase[d] && s < ibase[d] + nint[d]) { l = (uint32_t)d; v = first[d] + count[d] + (s - ibase[d]); }
+    for (int d = 1; d < T.max_len; ++d)
+      if (s >= T.ibase[d] && s < T.ibase[d] + T.nint[d]) { l = (uint32_t)d; v = T.first[d] + T.count[d] + (s - T.ibase[d]); }
     v = 2 * v + bit;
     ++l;
-    const uint32_t r = v - first[l];
-    if (r < count[l]) { *sym = sorted[base[l] + r]; return 0; }
-    if ((int)l >= max_len) return kErr;
-    return ibase[l] + (v - first[l] - count[l]);
+    const uint32_t r = v - T.first[l];
+    if (r < T.count[l]) { *sym = T.sorted[T.base[l] + r]; return 0; }
+    if ((int)l >= T.max_len) return err;
+    return T.ibase[l] + (v - T.first[l] - T.count[l]);
   };
   uint32_t* t = static_cast<uint32_t*>(h_table);
   for (uint32_t s = 0; s < 256; ++s)
     for (uint32_t nib = 0; nib < 16; ++nib) {
       uint32_t node = s, syms = 0, k = 0;
-      for (int i = 3; i >= 0 && node != kErr; --i) {
+      for (int i = 3; i >= 0 && node != err; --i) {
         int sym;
         node = step(node, (nib >> i) & 1u, &sym);
         if (sym >= 0) syms |= (uint32_t)sym << (8 * k++);
       }
-      const bool err = node == kErr;
-      t[2 * (s * 16 + nib)] = err ? 0 : syms;
-      t[2 * (s * 16 + nib) + 1] = err ? (kErr << 4) : ((node << 4) | ((8 * k) << 12));
+      const bool bad = node == err;
+      t[2 * (s * 16 + nib)] = bad ? 0 : syms;
+      t[2 * (s * 16 + nib) + 1] = bad ? (err << 7) : ((node << 7) | ((8 * k) << 16));
     }
   return ECF8_OK;
 }

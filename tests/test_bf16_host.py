@@ -85,8 +85,9 @@ def test_blob_info_rejects_damaged_headers():
 
 
 def _table(info):
-    t = L.bf16_table(info).view(np.uint32).reshape(256 * 16, 2)
-    return t[:, 0].astype(np.uint64), t[:, 1].astype(np.uint64)
+    """(exponents, count, next node) per entry, and the error node."""
+    t = L.bf16_table(info).view(np.uint32).reshape(256 * 16, 2).astype(np.int64)
+    return t[:, 0], (t[:, 1] >> 16) // 8, (t[:, 1] >> 7) & 0xFF, L.bf16_table_nodes(info)
 
 
 def _stream_bits(blob, hd):
@@ -100,17 +101,16 @@ def test_table_walk_decodes_the_whole_stream(name):
     x = CASES[name]
     blob = oracle.bf16_encode(x)
     hd = oracle.bf16_blob_header(blob)
-    syms, nxt = _table(L.bf16_blob_info(blob))
+    syms, cnt, nxt, err = _table(L.bf16_blob_info(blob))
     bits = _stream_bits(blob, hd)
     bits = np.concatenate([bits, np.zeros((-bits.size) % 4, np.uint8)])
     nibs = bits.reshape(-1, 4) @ np.array([8, 4, 2, 1])
     node, out = 0, []
     for v in nibs:
         e = node * 16 + int(v)
-        k = int(nxt[e] >> 12) // 8
-        out += [(int(syms[e]) >> (8 * j)) & 0xFF for j in range(k)]
-        node = int(nxt[e] >> 4) & 0xFF
-        assert node != 255
+        out += [(int(syms[e]) >> (8 * j)) & 0xFF for j in range(int(cnt[e]))]
+        node = int(nxt[e])
+        assert node != err
     lmin = int(hd["lengths"][hd["lengths"] > 0].min())
     pad = (-hd["code_bits"]) % 4  # zero bits after the stream decode as the all-zeros code
     extra = pad // lmin
@@ -118,25 +118,35 @@ def test_table_walk_decodes_the_whole_stream(name):
     assert np.array_equal(np.array(out[:x.size], dtype=np.uint16), (x >> 7) & 0xFF)
 
 
+def test_table_node_count_is_the_internal_nodes():
+    """A complete code over k exponents has k - 1 internal nodes."""
+    for name in ("normal", "random_bits", "two_symbols", "skewed_capped"):
+        info = L.bf16_blob_info(oracle.bf16_encode(CASES[name]))
+        assert L.bf16_table_nodes(info) == int((info.lengths > 0).sum()) - 1
+
+
 def test_table_error_node_and_invalid_bits():
     x = CASES["single_symbol"]
     info = L.bf16_blob_info(oracle.bf16_encode(x))
-    syms, nxt = _table(info)
-    assert int(nxt[0 * 16 + 0] >> 12) == 32 and int(syms[0]) == 0x80808080  # four 0-bit codes of exponent 128
+    syms, cnt, nxt, err = _table(info)
+    assert err == 1  # the root is the only node
+    assert cnt[0] == 4 and syms[0] == 0x80808080 and nxt[0] == 0  # four 1-bit codes 0 of exponent 128
     for v in range(1, 16):
-        assert (int(nxt[v]) >> 4) & 0xFF == 255  # a 1 bit is no code
-    assert all((int(nxt[255 * 16 + v]) >> 4) & 0xFF == 255 for v in range(16))  # the error node absorbs
+        assert nxt[v] == err and cnt[v] == 0  # a 1 bit is no code
+    for s_ in range(err, 256):
+        assert (nxt[16 * s_:16 * s_ + 16] == err).all()  # the error node (and the unused ones) absorb
     # a single exponent with a 3-bit code: one exponent per three zero bits
     ln = np.zeros(256, np.uint8)
     ln[128] = 3
     blob = oracle.bf16_encode(x, lengths=ln)
     assert np.array_equal(oracle.bf16_decode(blob, x.size), x)
-    syms, nxt = _table(L.bf16_blob_info(blob))
+    syms, cnt, nxt, err = _table(L.bf16_blob_info(blob))
+    assert err == 3
     node, got = 0, 0
     for _ in range(6):  # 24 zero bits = 8 codes
         e = node * 16
-        got += int(nxt[e] >> 12) // 8
-        node = int(nxt[e] >> 4) & 0xFF
+        got += int(cnt[e])
+        node = int(nxt[e])
     assert got == 8 and node == 0
 
 
@@ -147,7 +157,7 @@ def _emulate_kernel(blob, x_size):
     16-aligned base, then join with the kept bytes."""
     hd = oracle.bf16_blob_header(blob)
     info = L.bf16_blob_info(blob)
-    syms, nxt = _table(info)
+    syms, cnt_t, nxt, err = _table(info)
     lens = hd["lengths"]
     lmin = int(lens[lens > 0].min())
     gaps_b = blob[hd["gaps_off"]:hd["groups_off"]]
@@ -182,10 +192,9 @@ def _emulate_kernel(blob, x_size):
             for j in range(68):
                 v = int(bits[4 * j:4 * j + 4] @ np.array([8, 4, 2, 1]))
                 e = node * 16 + v
-                k = int(nxt[e] >> 12) // 8
-                got += [(int(syms[e]) >> (8 * q)) & 0xFF for q in range(k)]
-                node = int(nxt[e] >> 4) & 0xFF
-            assert node != 255 and len(got) <= 4 * 69
+                got += [(int(syms[e]) >> (8 * q)) & 0xFF for q in range(int(cnt_t[e]))]
+                node = int(nxt[e])
+            assert node != err and len(got) <= 4 * 69
             extra = (272 - E) // lmin
             assert len(got) >= extra
             cnt = len(got) - extra
@@ -211,3 +220,54 @@ def test_kernel_plan_emulation_reproduces_the_input(name):
     x = CASES[name][:12_000]
     blob = oracle.bf16_encode(x)
     assert np.array_equal(_emulate_kernel(blob, x.size), x)
+
+
+def _layout(info):
+    """The decoder's table layout for a code: wide when a 1-bit code exists,
+    else byte steps when the tree has at most 31 nodes, else narrow."""
+    lens = info.lengths
+    want = "wide" if lens[lens > 0].min() == 1 else "byte" if L.bf16_table_nodes(info) + 1 <= 32 else "narrow"
+    assert L.bf16_auto_layout(info) == want
+    return want
+
+
+@pytest.mark.parametrize("name", ["normal", "random_bits", "skewed_capped", "two_symbols"])
+def test_narrow_entries_hold_at_most_two_exponents(name):
+    """With no 1-bit code a nibble ends at most two codes, so the narrow
+    32-bit entry (16 bits of exponents, node, 8 x count <= 16) loses nothing."""
+    info = L.bf16_blob_info(oracle.bf16_encode(CASES[name]))
+    syms, cnt, nxt, err = _table(info)
+    live = slice(0, 16 * (err + 1))
+    if _layout(info) == "wide":
+        assert cnt[live].max() <= 4
+    else:
+        assert cnt[live].max() <= 2 and (syms[live] >> 16 == 0).all() and nxt[live].max() <= err
+
+
+def test_gpu_cases_cover_every_table_layout():
+    r = np.random.default_rng(5)
+    seen = {
+        _layout(L.bf16_blob_info(oracle.bf16_encode(x)))
+        for x in (CASES["normal"], CASES["random_bits"], CASES["two_symbols"], CASES["skewed_capped"],
+                  _bf16_bits(r.standard_normal(50_000) * np.exp(r.uniform(-60, 60, 50_000))))
+    }
+    assert seen == {"wide", "narrow", "byte"}
+
+
+@pytest.mark.parametrize("name", ["normal", "two_symbols", "skewed_capped"])
+def test_byte_steps_compose_two_nibble_steps(name):
+    """The byte-step entry the device builds for (node, byte) is the nibble
+    walk of the byte's high then low nibble: at most 4 exponents when no code
+    has 1 bit (a byte then ends at most 1 + 3 // 2 + ... codes)."""
+    info = L.bf16_blob_info(oracle.bf16_encode(CASES[name]))
+    syms, cnt, nxt, err = _table(info)
+    lens = info.lengths
+    for node in range(err + 1):
+        for byte in range(256):
+            e1 = node * 16 + (byte >> 4)
+            e2 = int(nxt[e1]) * 16 + (byte & 15)
+            k = int(cnt[e1]) + int(cnt[e2])
+            if lens[lens > 0].min() >= 2:
+                assert k <= 4
+            got = (int(syms[e1]) | (int(syms[e2]) << (8 * int(cnt[e1])))) & ((1 << 32) - 1)
+            assert got >> (8 * k) == 0 or k == 4

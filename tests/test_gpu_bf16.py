@@ -20,7 +20,7 @@ def env(gpu_available):
     return L, torch
 
 
-def _decode(env, blob, guard=64):
+def _decode(env, blob, guard=64, layout="auto"):
     L, torch = env
     info = L.bf16_blob_info(blob)
     d_blob = torch.from_numpy(blob).cuda()
@@ -28,7 +28,7 @@ def _decode(env, blob, guard=64):
     buf = torch.full((info.n + 2 * guard,), 0x5A5A, dtype=torch.int16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     launches = L.launch_count()
-    L.bf16_decode(info, d_blob, d_table, buf[guard:guard + info.n], status)
+    L.bf16_decode(info, d_blob, d_table, buf[guard:guard + info.n], status, layout=layout)
     torch.cuda.synchronize()
     if info.n:
         assert L.launch_count() == launches + 1
@@ -72,13 +72,58 @@ def test_decode_matches_the_oracle(env, name):
     assert np.array_equal(got, x)
 
 
+def _layouts(L, blob):
+    """Every table layout that can hold the blob's code."""
+    info = L.bf16_blob_info(blob)
+    lens = info.lengths
+    if lens[lens > 0].min() == 1:
+        return ["wide"]
+    small = L.bf16_table_nodes(info) + 1 <= 32
+    return ["wide", "narrow"] + (["narrow_lane", "byte"] if small else [])
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_every_table_layout_gives_the_same_output(env, name):
+    L, torch = env
+    x = CASES[name]
+    blob = oracle.bf16_encode(x)
+    want = oracle.bf16_decode(blob, x.size)
+    for layout in _layouts(L, blob):
+        got, status, intact = _decode(env, blob, layout=layout)
+        assert status == 0 and intact, layout
+        assert np.array_equal(got, want), layout
+
+
+def test_a_layout_that_cannot_hold_the_code_is_refused(env):
+    L, torch = env
+    blob = oracle.bf16_encode(CASES["two_symbols"])  # 1-bit codes: wide only
+    info = L.bf16_blob_info(blob)
+    d_blob = torch.from_numpy(blob).cuda()
+    d_table = torch.from_numpy(L.bf16_table(info)).cuda()
+    out = torch.empty(info.n, dtype=torch.int16, device="cuda")
+    for layout in ("narrow", "narrow_lane", "byte"):
+        with pytest.raises(L.Ecf8Error) as e:
+            L.bf16_decode(info, d_blob, d_table, out, layout=layout)
+        assert e.value.code == -6
+    blob = oracle.bf16_encode(CASES["random_bits"])  # 255 nodes: no lane-private or byte table
+    info = L.bf16_blob_info(blob)
+    for layout in ("narrow_lane", "byte"):
+        with pytest.raises(L.Ecf8Error) as e:
+            L.bf16_decode(info, torch.from_numpy(blob).cuda(), torch.from_numpy(L.bf16_table(info)).cuda(),
+                          torch.empty(info.n, dtype=torch.int16, device="cuda"), layout=layout)
+        assert e.value.code == -6
+
+
 @pytest.mark.parametrize("n", [1, 2, 15, 16, 17, 31, 33, 1000, 4095, 8191, 8192, 8193, 65_537])
 def test_small_and_ragged_sizes(env, n):
+    L, torch = env
     x = synth.llama3_8b_layer_bf16().tensors[2].generate_bf16(begin=n, count=n)
     blob = oracle.bf16_encode(x)
-    got, status, intact = _decode(env, blob)
-    assert status == 0 and intact
-    assert np.array_equal(got, oracle.bf16_decode(blob, n))
+    want = oracle.bf16_decode(blob, n)
+    for layout in _layouts(L, blob):
+        got, status, intact = _decode(env, blob, layout=layout)
+        assert status == 0 and intact, layout
+        assert np.array_equal(got, want), layout
 
 
 @pytest.mark.parametrize("cap", [8, 12])
@@ -171,7 +216,9 @@ def test_damaged_streams_are_reported_and_stay_in_bounds(env, seed):
     b[hd["groups_off"] + 8 * k:hd["groups_off"] + 8 * k + 8] = np.frombuffer(
         np.uint64(int(r.integers(0, 1 << 40))).tobytes(), np.uint8)
     kinds.append(b)
+    L = env[0]
     for bad in kinds:
-        got, status, intact = _decode(env, bad)
-        assert intact
-        assert status != 0 or np.array_equal(got, x)
+        for layout in _layouts(L, blob):
+            got, status, intact = _decode(env, bad, layout=layout)
+            assert intact, layout
+            assert status != 0 or np.array_equal(got, x), layout
