@@ -622,7 +622,10 @@ def run_bf16(args):
     def one(k, layout="auto"):  # on the current stream (the capture stream inside a graph)
         L.bf16_decode(infos[k], d_blobs[k], d_tables[k], d_outs[k], status, layout=layout)
 
-    def layer():
+    def layer():  # the layer's seven tensors in one batched launch
+        L.bf16_decode_batched([(infos[k], d_blobs[k], d_tables[k], d_outs[k]) for k in range(len(specs))], status)
+
+    def layer_separate():
         for k in range(len(specs)):
             one(k)
 
@@ -651,8 +654,9 @@ def run_bf16(args):
     peak, peak_kind = measured_hbm_peak()
     launches0 = L.launch_count()
     g_layer = graphed(layer, 1)
-    launches = L.launch_count() - launches0 - len(specs)  # the capture's launches (the warm call excluded)
+    launches = (L.launch_count() - launches0) // 2  # the warm call's and the capture's
     ms = _time_launches(torch, g_layer.replay, max(1, args.steps), args.warmup)
+    ms_separate = _time_launches(torch, graphed(layer_separate, 1).replay, max(1, args.steps), args.warmup)
     per = []
     for k, spec in enumerate(specs):
         g_one = graphed(lambda: one(k), 10)
@@ -680,10 +684,11 @@ def run_bf16(args):
             "compressed_bytes": blob, "ratio_vs_bf16": round(2 * n / blob, 4),
             "bits_per_weight": round(8 * blob / n, 4), "ms_per_layer": round(ms, 5),
             "gbps_bf16_out": round(2 * n / ms / 1e6, 2), "gpu_launches_per_layer": launches,
+            "ms_per_layer_one_launch_per_tensor": round(ms_separate, 5),
             "roofline": {"bound": "hbm", "achieved": round(alg / ms / 1e6, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(alg / ms / 1e6 / peak, 4),
                          "algorithmic_bytes": alg, "peak_source": f"{peak_kind} hbm_gbs"},
-            "timing": "CUDA graph of the layer's 7 launches, replayed; per tensor: graph of 10 launches "
+            "timing": "CUDA graph of the layer's batched launch, replayed; per tensor: graph of 10 launches "
                       "(tensors whose blob + output fit in L2 run L2-warm there)",
             "l2": "inputs+outputs larger than L2 (no flush)", "per_tensor": per,
             "auto_layout": {spec.name: L.bf16_auto_layout(i) for spec, i in zip(specs, infos)},

@@ -373,6 +373,23 @@ int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, const void*
 #define ECF8_BF16_LAYOUT_NARROW_LANE 2
 #define ECF8_BF16_LAYOUT_BYTE 3
 
+/* One tensor of a batched BF16 decode (pointers as for ecf8_bf16_decode). */
+typedef struct ecf8_bf16_tensor {
+  const ecf8_bf16_info* info; /* host */
+  const void* d_blob;         /* device, 16-byte aligned */
+  const void* d_table;        /* device, 16-byte aligned, ecf8_bf16_build_table of info */
+  uint16_t* d_out;            /* device, 16-byte aligned, info->n elements */
+} ecf8_bf16_tensor;
+
+/* Tensors a batched launch carries in its parameters. */
+#define ECF8_BF16_BATCH_MAX 32
+
+/* Decode count BF16 blobs: one launch per table layout present (AUTO per
+ * tensor) and per ECF8_BF16_BATCH_MAX tensors, each CTA over a contiguous
+ * run of the tensors' groups.  Every tensor is checked before anything is
+ * enqueued (errors as ecf8_bf16_decode); empty tensors are skipped. */
+int ecf8_bf16_decode_batched(const ecf8_bf16_tensor* tensors, int count, int32_t* d_status, cudaStream_t stream);
+
 /* The layout ecf8_bf16_decode picks for info's code (>= 0), or an error. */
 int ecf8_bf16_auto_layout(const ecf8_bf16_info* info);
 

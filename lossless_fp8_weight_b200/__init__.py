@@ -127,6 +127,15 @@ _lib.ecf8_bf16_decode.argtypes = [ctypes.POINTER(Bf16Info), _p, _p, _p, _sz, _p,
 _lib.ecf8_bf16_decode_layout.argtypes = [ctypes.POINTER(Bf16Info), _p, _p, _p, _sz, _p, _p, _i32]
 _lib.ecf8_bf16_auto_layout.argtypes = [ctypes.POINTER(Bf16Info)]
 BF16_LAYOUTS = {"auto": -1, "wide": 0, "narrow": 1, "narrow_lane": 2, "byte": 3}
+BF16_BATCH_MAX = 32
+
+
+class Bf16Tensor(ctypes.Structure):
+    _fields_ = [("info", ctypes.POINTER(Bf16Info)), ("d_blob", ctypes.c_void_p), ("d_table", ctypes.c_void_p),
+                ("d_out", ctypes.c_void_p)]
+
+
+_lib.ecf8_bf16_decode_batched.argtypes = [ctypes.POINTER(Bf16Tensor), _i32, _p, _p]
 
 
 class LayerTensor(ctypes.Structure):
@@ -466,3 +475,13 @@ def bf16_decode(info: Bf16Info, d_blob, d_table, d_out, status=None, stream=None
     ``layout`` forces one of the decoder's table layouts (same output)."""
     _check(_lib.ecf8_bf16_decode_layout(ctypes.byref(info), _ptr(d_blob), _ptr(d_table), _ptr(d_out), info.n,
                                         _ptr(status), _stream(stream), BF16_LAYOUTS[layout]), "ecf8_bf16_decode")
+
+
+def bf16_decode_batched(items, status=None, stream=None) -> None:
+    """Asynchronously decode several BF16 blobs: ``items`` is a sequence of
+    (info, d_blob, d_table, d_out); one launch per table layout present."""
+    infos = [it[0] for it in items]
+    arr = (Bf16Tensor * max(1, len(items)))()
+    for k, (info, d_blob, d_table, d_out) in enumerate(items):
+        arr[k] = Bf16Tensor(ctypes.pointer(infos[k]), _ptr(d_blob), _ptr(d_table), _ptr(d_out))
+    _check(_lib.ecf8_bf16_decode_batched(arr, len(items), _ptr(status), _stream(stream)), "ecf8_bf16_decode_batched")

@@ -37,7 +37,10 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <string.h>
+
 #include <type_traits>
+#include <vector>
 
 #include "ecf8.h"
 #include "ecf8_format.h"
@@ -71,17 +74,28 @@ struct alignas(16) WarpArea {
   uint32_t stage[Cfg<V>::kStageWords];     // exponent byte i at byte i (from the group's 16-aligned base)
 };
 
+// One tensor of a launch.
 struct Args {
   const uint32_t* gaps;
   const uint64_t* groups;
   const uint32_t* stream;
   const uint8_t* kept;
   uint16_t* out;
+  const uint2* table;   // the host-built nibble table (device)
   uint64_t n, code_bits;
   uint32_t n_groups, lmin;
-  uint32_t nodes;     // tree nodes; the error node is node `nodes`
-  uint32_t zc_off, warp_off;
+  uint32_t nodes;       // tree nodes; the error node is node `nodes`
+  uint32_t group_base;  // groups of the launch's earlier tensors
 };
+
+// Up to ECF8_BF16_BATCH_MAX tensors of one table layout, in the launch's
+// parameters; their groups are numbered consecutively in tensor order.
+struct Batch {
+  Args t[ECF8_BF16_BATCH_MAX];
+  uint32_t count, total_groups;
+  uint32_t zc_off, warp_off;  // shared-memory offsets: zero-code table, warp areas
+};
+static_assert(sizeof(Batch) <= 4096, "kernel parameter block");
 
 struct GroupIn {
   uint32_t w[kWords + 1];
@@ -336,30 +350,26 @@ __device__ __forceinline__ uint32_t narrow_entry(uint2 w) {
   return (w.x & 0xFFFFu) | (((w.y >> 7) & 0xFFu) << 16) | (((w.y >> 16) & 0x1Fu) << 27);
 }
 
+// Tensor a's decode table and zero-code counts into shared memory (every
+// thread of the CTA takes part; the first warp area serves as scratch).
 template <int V>
-__global__ void __launch_bounds__(Cfg<V>::kMaxWarps * 32, 1)
-    decode_kernel(const uint2* __restrict__ d_table, Args a, int32_t* status) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  const uint32_t warps = blockDim.x >> 5, warp = threadIdx.x >> 5;
-  uint32_t g = blockIdx.x * warps + warp;
-  GroupIn in;
-  if (g < a.n_groups) fetch_group(a, g, in);  // in flight while the table is staged
-
+__device__ __forceinline__ void stage_table(const Args& a, uint8_t* smem, uint32_t zc_off, uint32_t warp_off) {
   const uint32_t entries = (a.nodes + 1) * 16;
+  const uint2* src = a.table;
   if (V == kWide) {
-    uint2* t = reinterpret_cast<uint2*>(smem_raw);
+    uint2* t = reinterpret_cast<uint2*>(smem);
 #pragma unroll 8
-    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) t[i] = __ldg(d_table + i);
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) t[i] = __ldg(src + i);
   } else if (V == kNarrow) {
-    uint32_t* t = reinterpret_cast<uint32_t*>(smem_raw);
+    uint32_t* t = reinterpret_cast<uint32_t*>(smem);
 #pragma unroll 8
-    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) t[i] = narrow_entry(__ldg(d_table + i));
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) t[i] = narrow_entry(__ldg(src + i));
   } else if (V == kByte) {
-    // the nibble entries once into the first warp area, then two of them per (node, byte)
-    uint2* once = reinterpret_cast<uint2*>(smem_raw + a.warp_off);
-    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) once[i] = __ldg(d_table + i);
+    // the nibble entries once into scratch, then two of them per (node, byte)
+    uint2* once = reinterpret_cast<uint2*>(smem + warp_off);
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) once[i] = __ldg(src + i);
     __syncthreads();
-    uint2* t = reinterpret_cast<uint2*>(smem_raw);
+    uint2* t = reinterpret_cast<uint2*>(smem);
     for (uint32_t i = threadIdx.x; i < (a.nodes + 1) * 256; i += blockDim.x) {
       const uint32_t node = i >> 8, byte = i & 255;
       const uint2 e1 = once[node * 16 + (byte >> 4)];
@@ -369,25 +379,50 @@ __global__ void __launch_bounds__(Cfg<V>::kMaxWarps * 32, 1)
       t[i] = make_uint2(e1.x | (c1 < 32 ? e2.x << c1 : 0u), (n2 << 11) | ((c1 + c2) << 24));
     }
   } else {
-    // each entry read once into the first warp area, then copied to every lane's slot
-    uint32_t* once = reinterpret_cast<uint32_t*>(smem_raw + a.warp_off);
-    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) once[i] = narrow_entry(__ldg(d_table + i));
+    // each entry read once into scratch, then copied to every lane's slot
+    uint32_t* once = reinterpret_cast<uint32_t*>(smem + warp_off);
+    for (uint32_t i = threadIdx.x; i < entries; i += blockDim.x) once[i] = narrow_entry(__ldg(src + i));
     __syncthreads();
-    uint32_t* t = reinterpret_cast<uint32_t*>(smem_raw);
+    uint32_t* t = reinterpret_cast<uint32_t*>(smem);
     for (uint32_t i = threadIdx.x; i < entries * 32; i += blockDim.x) t[i] = once[i >> 5];
   }
-  uint16_t* zero_codes = reinterpret_cast<uint16_t*>(smem_raw + a.zc_off);
+  uint16_t* zero_codes = reinterpret_cast<uint16_t*>(smem + zc_off);
   for (int z = threadIdx.x; z <= kPadBits; z += blockDim.x) zero_codes[z] = (uint16_t)(z / a.lmin);
-  __syncthreads();
-  WarpArea<V>* wa = reinterpret_cast<WarpArea<V>*>(smem_raw + a.warp_off) + warp;
-  if (g >= a.n_groups) return;
-  for (; g < a.n_groups; g += gridDim.x * warps) {
-    GroupIn nx;
-    const uint32_t gn = g + gridDim.x * warps;
-    const bool more = gn < a.n_groups;
-    if (more) fetch_group(a, gn, nx);
-    process_group<V>(a, g, in, smem_raw, zero_codes, wa, status);
-    if (more) in = nx;
+}
+
+// Persistent CTAs, each over a contiguous run of the batch's groups.  The run
+// is cut at tensor boundaries into segments; for each segment the CTA stages
+// that tensor's table, then its warps take the segment's groups in turn, each
+// fetching its next group's stream slice while it decodes the current one.
+template <int V>
+__global__ void __launch_bounds__(Cfg<V>::kMaxWarps * 32, 1)
+    decode_kernel(const __grid_constant__ Batch b, int32_t* status) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t warps = blockDim.x >> 5, warp = threadIdx.x >> 5;
+  const uint32_t g_begin = (uint32_t)((uint64_t)b.total_groups * blockIdx.x / gridDim.x);
+  const uint32_t g_end = (uint32_t)((uint64_t)b.total_groups * (blockIdx.x + 1) / gridDim.x);
+  const uint16_t* zero_codes = reinterpret_cast<const uint16_t*>(smem_raw + b.zc_off);
+  WarpArea<V>* wa = reinterpret_cast<WarpArea<V>*>(smem_raw + b.warp_off) + warp;
+  uint32_t k = 0;
+  for (uint32_t seg = g_begin; seg < g_end;) {
+    while (k + 1 < b.count && b.t[k + 1].group_base <= seg) ++k;
+    const Args& a = b.t[k];
+    const uint32_t seg_end = min(g_end, a.group_base + a.n_groups);
+    uint32_t g = seg + warp;
+    GroupIn in;
+    if (g < seg_end) fetch_group(a, g - a.group_base, in);  // in flight while the table is staged
+    __syncthreads();  // the previous segment's warps are done with the table
+    stage_table<V>(a, smem_raw, b.zc_off, b.warp_off);
+    __syncthreads();
+    for (; g < seg_end; g += warps) {
+      GroupIn nx;
+      const uint32_t gn = g + warps;
+      const bool more = gn < seg_end;
+      if (more) fetch_group(a, gn - a.group_base, nx);
+      process_group<V>(a, g - a.group_base, in, smem_raw, zero_codes, wa, status);
+      if (more) in = nx;
+    }
+    seg = seg_end;
   }
 }
 
@@ -395,29 +430,58 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 uint32_t up16(uint32_t x) { return (x + 15) & ~15u; }
 
 template <int V>
-int launch(Args a, const void* d_table, int32_t* d_status, cudaStream_t s) {
-  const uint32_t entries = (a.nodes + 1) * 16;
-  const uint32_t table_bytes = V == kWide ? entries * 8 : V == kNarrow ? entries * 4
-                               : V == kNarrowLane ? entries * 128 : (a.nodes + 1) * 2048;
-  a.zc_off = table_bytes;
-  a.warp_off = up16(a.zc_off + 2 * (kPadBits + 1));
+uint32_t table_bytes(uint32_t nodes) {
+  const uint32_t entries = (nodes + 1) * 16;
+  return V == kWide ? entries * 8 : V == kNarrow ? entries * 4 : V == kNarrowLane ? entries * 128 : (nodes + 1) * 2048;
+}
+
+// One launch over ts[0, count) (count <= ECF8_BF16_BATCH_MAX, every tensor
+// non-empty and holdable by layout V).
+template <int V>
+int launch(const Args* ts, uint32_t count, int32_t* d_status, cudaStream_t s) {
+  Batch b;
+  memset(&b, 0, sizeof(b));
+  uint64_t total = 0;
+  uint32_t tbytes = 0;
+  for (uint32_t i = 0; i < count; ++i) {
+    b.t[i] = ts[i];
+    b.t[i].group_base = (uint32_t)total;
+    total += ts[i].n_groups;
+    const uint32_t tb = table_bytes<V>(ts[i].nodes);
+    tbytes = tb > tbytes ? tb : tbytes;
+  }
+  if (total == 0) return ECF8_OK;
+  if (total > 0xFFFFFFFFull) return ECF8_ERR_ARG;
+  b.count = count;
+  b.total_groups = (uint32_t)total;
+  b.zc_off = tbytes;
+  b.warp_off = up16(b.zc_off + 2 * (kPadBits + 1));
   int dev = 0, sms = 0, smem_max = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
       cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev))
     return ECF8_ERR_CUDA;
-  if ((uint32_t)smem_max <= a.warp_off) return ECF8_ERR_UNSUPPORTED;
-  const uint32_t fit = ((uint32_t)smem_max - a.warp_off) / (uint32_t)sizeof(WarpArea<V>);
+  if ((uint32_t)smem_max <= b.warp_off) return ECF8_ERR_UNSUPPORTED;
+  const uint32_t fit = ((uint32_t)smem_max - b.warp_off) / (uint32_t)sizeof(WarpArea<V>);
   const uint32_t warps = fit < (uint32_t)Cfg<V>::kMaxWarps ? fit : (uint32_t)Cfg<V>::kMaxWarps;
   if (warps == 0) return ECF8_ERR_UNSUPPORTED;
-  const uint32_t smem = a.warp_off + warps * (uint32_t)sizeof(WarpArea<V>);
+  const uint32_t smem = b.warp_off + warps * (uint32_t)sizeof(WarpArea<V>);
   if (cudaFuncSetAttribute(decode_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max))
     return ECF8_ERR_CUDA;
-  const uint64_t ctas_needed = ((uint64_t)a.n_groups + warps - 1) / warps;
+  const uint64_t ctas_needed = (total + warps - 1) / warps;
   const uint32_t grid = (uint32_t)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
-  decode_kernel<V><<<grid, warps * 32, smem, s>>>(static_cast<const uint2*>(d_table), a, d_status);
+  decode_kernel<V><<<grid, warps * 32, smem, s>>>(b, d_status);
   if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
   ecf8::note_launch();
   return ECF8_OK;
+}
+
+int launch_layout(int layout, const Args* ts, uint32_t count, int32_t* d_status, cudaStream_t s) {
+  switch (layout) {
+    case kWide: return launch<kWide>(ts, count, d_status, s);
+    case kNarrow: return launch<kNarrow>(ts, count, d_status, s);
+    case kNarrowLane: return launch<kNarrowLane>(ts, count, d_status, s);
+    default: return launch<kByte>(ts, count, d_status, s);
+  }
 }
 
 }  // namespace
@@ -457,44 +521,75 @@ extern "C" int ecf8_bf16_auto_layout(const ecf8_bf16_info* info) {
   return nodes + 1 <= 32 ? kByte : kNarrow;
 }
 
-extern "C" int ecf8_bf16_decode_layout(const ecf8_bf16_info* info, const void* d_blob, const void* d_table,
-                                       uint16_t* d_out, size_t n, int32_t* d_status, cudaStream_t s, int layout) {
-  if (!info || n != info->n) return ECF8_ERR_ARG;
+namespace ecf8_bf16 {
+namespace {
+
+// Checks one tensor and fills its launch arguments; resolves AUTO.
+int prepare(const ecf8_bf16_tensor& t, int* layout, Args* a) {
+  const ecf8_bf16_info* info = t.info;
+  if (!info) return ECF8_ERR_ARG;
   if (info->chunk_bytes != (uint32_t)kC || info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
-  if (n == 0) return ECF8_OK;
-  if (layout == ECF8_BF16_LAYOUT_AUTO) {
-    const int l = ecf8_bf16_auto_layout(info);
-    if (l < 0) return l;
-    layout = l;
-  }
-  if (!d_blob || !d_table || !d_out) return ECF8_ERR_ARG;
-  if (!aligned16(d_blob) || !aligned16(d_table) || !aligned16(d_out)) return ECF8_ERR_ALIGN;
+  if (info->n == 0) return ECF8_OK;
+  if (!t.d_blob || !t.d_table || !t.d_out) return ECF8_ERR_ARG;
+  if (!aligned16(t.d_blob) || !aligned16(t.d_table) || !aligned16(t.d_out)) return ECF8_ERR_ALIGN;
   const uint32_t nodes = ecf8_bf16_table_nodes(info);
   if (nodes == 0) return ECF8_ERR_CODEBOOK;
   const uint32_t lmin = shortest(info);
-  if (!layout_holds(layout, lmin, nodes)) return ECF8_ERR_UNSUPPORTED;
-  const uint8_t* b = static_cast<const uint8_t*>(d_blob);
+  if (*layout == ECF8_BF16_LAYOUT_AUTO) *layout = lmin == 1 ? kWide : nodes + 1 <= 32 ? kByte : kNarrow;
+  if (!layout_holds(*layout, lmin, nodes)) return ECF8_ERR_UNSUPPORTED;
+  const uint8_t* b = static_cast<const uint8_t*>(t.d_blob);
+  a->gaps = reinterpret_cast<const uint32_t*>(b + info->gaps_off);
+  a->groups = reinterpret_cast<const uint64_t*>(b + info->groups_off);
+  a->stream = reinterpret_cast<const uint32_t*>(b + info->stream_off);
+  a->kept = b + info->kept_off;
+  a->out = t.d_out;
+  a->table = static_cast<const uint2*>(t.d_table);
+  a->n = info->n;
+  a->code_bits = info->code_bits;
+  a->n_groups = info->n_groups;
+  a->lmin = lmin;
+  a->nodes = nodes;
+  a->group_base = 0;
+  return ECF8_OK;
+}
+
+}  // namespace
+}  // namespace ecf8_bf16
+
+extern "C" int ecf8_bf16_decode_layout(const ecf8_bf16_info* info, const void* d_blob, const void* d_table,
+                                       uint16_t* d_out, size_t n, int32_t* d_status, cudaStream_t s, int layout) {
+  if (!info || n != info->n) return ECF8_ERR_ARG;
+  if (layout < ECF8_BF16_LAYOUT_AUTO || layout > ECF8_BF16_LAYOUT_BYTE) return ECF8_ERR_ARG;
+  const ecf8_bf16_tensor t = {info, d_blob, d_table, d_out};
   Args a;
-  a.gaps = reinterpret_cast<const uint32_t*>(b + info->gaps_off);
-  a.groups = reinterpret_cast<const uint64_t*>(b + info->groups_off);
-  a.stream = reinterpret_cast<const uint32_t*>(b + info->stream_off);
-  a.kept = b + info->kept_off;
-  a.out = d_out;
-  a.n = info->n;
-  a.code_bits = info->code_bits;
-  a.n_groups = info->n_groups;
-  a.lmin = lmin;
-  a.nodes = nodes;
-  a.zc_off = a.warp_off = 0;
-  switch (layout) {
-    case kWide: return launch<kWide>(a, d_table, d_status, s);
-    case kNarrow: return launch<kNarrow>(a, d_table, d_status, s);
-    case kNarrowLane: return launch<kNarrowLane>(a, d_table, d_status, s);
-    default: return launch<kByte>(a, d_table, d_status, s);
-  }
+  const int rc = prepare(t, &layout, &a);
+  if (rc != ECF8_OK || n == 0) return rc;
+  return launch_layout(layout, &a, 1, d_status, s);
 }
 
 extern "C" int ecf8_bf16_decode(const ecf8_bf16_info* info, const void* d_blob, const void* d_table, uint16_t* d_out,
                                 size_t n, int32_t* d_status, cudaStream_t s) {
   return ecf8_bf16_decode_layout(info, d_blob, d_table, d_out, n, d_status, s, ECF8_BF16_LAYOUT_AUTO);
+}
+
+extern "C" int ecf8_bf16_decode_batched(const ecf8_bf16_tensor* tensors, int count, int32_t* d_status,
+                                        cudaStream_t s) {
+  if (count < 0 || (count > 0 && !tensors)) return ECF8_ERR_ARG;
+  // every tensor checked before anything is enqueued
+  std::vector<Args> by_layout[4];
+  for (int i = 0; i < count; ++i) {
+    int layout = ECF8_BF16_LAYOUT_AUTO;
+    Args a;
+    const int rc = prepare(tensors[i], &layout, &a);
+    if (rc != ECF8_OK) return rc;
+    if (tensors[i].info->n) by_layout[layout].push_back(a);
+  }
+  for (int l = 0; l < 4; ++l)
+    for (size_t i = 0; i < by_layout[l].size(); i += ECF8_BF16_BATCH_MAX) {
+      const size_t c = by_layout[l].size() - i < (size_t)ECF8_BF16_BATCH_MAX ? by_layout[l].size() - i
+                                                                              : (size_t)ECF8_BF16_BATCH_MAX;
+      const int rc = launch_layout(l, by_layout[l].data() + i, (uint32_t)c, d_status, s);
+      if (rc != ECF8_OK) return rc;
+    }
+  return ECF8_OK;
 }

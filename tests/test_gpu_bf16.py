@@ -161,6 +161,65 @@ def test_full_llama3_8b_layer(env):
         assert np.array_equal(got, x)
 
 
+def _batched(env, blobs, guard=64):
+    L, torch = env
+    infos = [L.bf16_blob_info(b) for b in blobs]
+    keep, items, bufs = [], [], []
+    for info, blob in zip(infos, blobs):
+        d_blob = torch.from_numpy(blob).cuda()
+        d_table = torch.from_numpy(L.bf16_table(info)).cuda()
+        buf = torch.full((info.n + 2 * guard,), 0x5A5A, dtype=torch.int16, device="cuda")
+        keep += [d_blob, d_table]
+        bufs.append(buf)
+        items.append((info, d_blob, d_table, buf[guard:guard + info.n]))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    launches = L.launch_count()
+    L.bf16_decode_batched(items, status)
+    torch.cuda.synchronize()
+    outs = []
+    for info, buf in zip(infos, bufs):
+        got = buf.cpu().numpy().view(np.uint16)
+        assert (got[:guard] == 0x5A5A).all() and (got[guard + info.n:] == 0x5A5A).all()
+        outs.append(got[guard:guard + info.n])
+    return outs, int(status.item()), L.launch_count() - launches
+
+
+def test_batched_mixed_layouts_and_an_empty_tensor(env):
+    L = env[0]
+    xs = list(CASES.values()) + [np.zeros(0, np.uint16)]
+    blobs = [oracle.bf16_encode(x) for x in xs]
+    outs, status, launches = _batched(env, blobs)
+    assert status == 0
+    assert launches == len({L.bf16_auto_layout(L.bf16_blob_info(b)) for b in blobs if x_size(b)})
+    for got, x, blob in zip(outs, xs, blobs):
+        assert np.array_equal(got, oracle.bf16_decode(blob, x.size))
+
+
+def x_size(blob):
+    return int(oracle.bf16_blob_header(blob)["n"])
+
+
+def test_batched_more_tensors_than_one_launch_carries(env):
+    L = env[0]
+    spec = synth.llama3_8b_layer_bf16().tensors[1]
+    xs = [spec.generate_bf16(begin=7919 * k, count=3000 + 977 * k) for k in range(L.BF16_BATCH_MAX + 9)]
+    blobs = [oracle.bf16_encode(x) for x in xs]
+    outs, status, launches = _batched(env, blobs)
+    assert status == 0 and launches == 2
+    for got, x in zip(outs, xs):
+        assert np.array_equal(got, x)
+
+
+def test_batched_full_llama3_8b_layer(env):
+    L = env[0]
+    xs = [t.generate_bf16() for t in synth.llama3_8b_layer_bf16().tensors]
+    blobs = [L.bf16_encode(x) for x in xs]
+    outs, status, launches = _batched(env, blobs)
+    assert status == 0 and launches == 1
+    for got, x in zip(outs, xs):
+        assert np.array_equal(got, x)
+
+
 def test_output_is_a_usable_bfloat16_tensor(env):
     L, torch = env
     w = torch.randn(4096, 1024, dtype=torch.float32).to(torch.bfloat16)
