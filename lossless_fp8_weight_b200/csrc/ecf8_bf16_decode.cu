@@ -28,9 +28,9 @@
 //    reads its own bank and a lookup is one shared-memory wavefront;
 //  - byte: shortest code >= 2 bits and at most 31 nodes: one entry per
 //    (node, byte), composed on the device from two nibble entries (a byte
-//    ends at most 4 codes: 64-bit entries {exponents, node << 11 | 8 count
-//    << 24}), so a lane walks 34 steps instead of 68 (the default for such
-//    codes: half the table steps, at the price of bank conflicts).
+//    ends at most 4 codes: 64-bit entries {exponents, node << 11 | (node &
+//    15) << 3 | 8 count << 24}, slots swizzled across the bank pairs), so a
+//    lane walks 34 steps instead of 68 (the default for such codes).
 // Corrupt input is reported through the status word; no access leaves its
 // buffer and no loop runs without a bound.
 #include <cuda_runtime.h>
@@ -197,16 +197,27 @@ struct Walker<kWide> {
   __device__ __forceinline__ uint32_t node() const { return (y >> 7) & 0xFFu; }
 };
 
+// Byte-table slot of (node, byte): the low 4 bits of the byte index are
+// XORed with its high nibble and the node's low 4 bits (a bijection within the
+// node's 256 entries), so that the 8-byte entries the lanes of a warp read
+// spread over the bank pairs by the whole byte and node, not by the byte's low
+// nibble alone.
+__host__ __device__ __forceinline__ uint32_t byte_slot(uint32_t node, uint32_t byte) {
+  return node * 256 + ((byte & 0xF0u) | ((byte ^ (byte >> 4) ^ node) & 15u));
+}
+
 template <>
 struct Walker<kByte> {
-  // entry (node, byte) at byte offset node * 2048 + byte * 8
+  // entry (node, byte) at byte offset 8 * byte_slot(node, byte); y carries
+  // node << 11 | (node & 15) << 3, so one LOP3 gives the next slot's offset
   static constexpr int kSteps = kNibbles / 2;
   const uint8_t* table;
   uint32_t y = 0;
   __device__ __forceinline__ Walker(const uint8_t* t, uint32_t) : table(t) {}
   __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
-    const uint32_t byte = (sw[j >> 2] >> (24 - 8 * (j & 3))) & 0xFFu;
-    const uint2 e = *reinterpret_cast<const uint2*>(table + ((y & (0x1Fu << 11)) | (byte << 3)));
+    const uint32_t b8 = ((sw[j >> 2] >> (24 - 8 * (j & 3))) & 0xFFu) << 3;
+    const uint32_t swz8 = b8 ^ ((b8 >> 4) & 0x78u);  // (byte & 0xF0 | (byte ^ byte >> 4) & 15) * 8
+    const uint2 e = *reinterpret_cast<const uint2*>(table + ((y & ((0x1Fu << 11) | (15u << 3))) ^ swz8));
     y = e.y;
     syms = e.x;
     bits8 = e.y >> 24;
@@ -376,7 +387,8 @@ __device__ __forceinline__ void stage_table(const Args& a, uint8_t* smem, uint32
       const uint32_t n1 = (e1.y >> 7) & 0xFFu, c1 = (e1.y >> 16) & 0x3Fu;
       const uint2 e2 = once[(n1 <= a.nodes ? n1 : a.nodes) * 16 + (byte & 15)];
       const uint32_t n2 = n1 == a.nodes ? a.nodes : (e2.y >> 7) & 0xFFu, c2 = (e2.y >> 16) & 0x3Fu;
-      t[i] = make_uint2(e1.x | (c1 < 32 ? e2.x << c1 : 0u), (n2 << 11) | ((c1 + c2) << 24));
+      t[byte_slot(node, byte)] =
+          make_uint2(e1.x | (c1 < 32 ? e2.x << c1 : 0u), (n2 << 11) | ((n2 & 15u) << 3) | ((c1 + c2) << 24));
     }
   } else {
     // each entry read once into scratch, then copied to every lane's slot
