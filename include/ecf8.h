@@ -319,13 +319,15 @@ typedef struct ecf8_bf16_info {
 int ecf8_bf16_code_lengths(const uint16_t* x, size_t n, uint32_t max_len, uint8_t len[256]);
 
 /* Exact blob size for x under len.  ECF8_ERR_CODEBOOK if an exponent of x has
- * no code. */
+ * no code, or if len is not a complete prefix code of at most 16 bits (a
+ * single present value may have any length). */
 int ecf8_bf16_encoded_size(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,
                            uint32_t group_chunks, size_t* bytes);
 
 /* Encode n BF16 bit patterns into blob (host, capacity cap); the bytes are
- * those of the oracle's encoder for the same lengths.  ECF8_ERR_CAPACITY if
- * cap is short; *bytes gets the size. */
+ * those of the oracle's encoder for the same lengths.  ECF8_ERR_CODEBOOK as
+ * for ecf8_bf16_encoded_size; ECF8_ERR_CAPACITY if cap is short; *bytes gets
+ * the size. */
 int ecf8_bf16_encode(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,
                      uint32_t group_chunks, void* blob, size_t cap, size_t* bytes);
 

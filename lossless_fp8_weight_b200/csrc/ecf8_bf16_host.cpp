@@ -116,6 +116,21 @@ bool package_merge(const uint64_t* h, int limit, uint8_t* len) {
   return true;
 }
 
+// The lengths the blob parser accepts: at most 16 bits, and a complete
+// prefix code (Kraft sum 1) unless a single value is present.
+bool valid_lengths(const uint8_t* len) {
+  uint64_t kraft = 0;
+  int present = 0;
+  for (int s = 0; s < kSym; ++s) {
+    if (len[s] > kMaxLen) return false;
+    if (len[s]) {
+      kraft += 1ull << (kMaxLen - len[s]);
+      ++present;
+    }
+  }
+  return present == 0 || (present == 1 ? kraft <= (1ull << kMaxLen) : kraft == (1ull << kMaxLen));
+}
+
 bool canonical(const uint8_t* len, uint32_t* code) {
   int count[kMaxLen + 2] = {0};
   uint32_t next[kMaxLen + 2] = {0};
@@ -150,6 +165,7 @@ int ecf8_bf16_code_lengths(const uint16_t* x, size_t n, uint32_t max_len, uint8_
 int ecf8_bf16_encoded_size(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,
                            uint32_t group_chunks, size_t* bytes) {
   if (!len || !bytes || (!x && n)) return ECF8_ERR_ARG;
+  if (!valid_lengths(len)) return ECF8_ERR_CODEBOOK;
   uint64_t bits = 0;
   for (size_t i = 0; i < n; ++i) {
     const uint8_t l = len[(x[i] >> 7) & 0xFF];
@@ -166,7 +182,7 @@ int ecf8_bf16_encode(const uint16_t* x, size_t n, const uint8_t len[256], uint32
                      uint32_t group_chunks, void* blob_v, size_t cap, size_t* bytes) {
   if (!len || !blob_v || !bytes || (!x && n)) return ECF8_ERR_ARG;
   uint32_t code[kSym];
-  if (!canonical(len, code)) return ECF8_ERR_CODEBOOK;
+  if (!valid_lengths(len) || !canonical(len, code)) return ECF8_ERR_CODEBOOK;
   uint64_t bits = 0;
   int max_len = 0;
   for (int s = 0; s < kSym; ++s) max_len = std::max<int>(max_len, len[s]);

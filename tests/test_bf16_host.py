@@ -271,3 +271,21 @@ def test_byte_steps_compose_two_nibble_steps(name):
                 assert k <= 4
             got = (int(syms[e1]) | (int(syms[e2]) << (8 * int(cnt[e1])))) & ((1 << 32) - 1)
             assert got >> (8 * k) == 0 or k == 4
+
+
+def test_encoder_refuses_lengths_that_are_not_a_complete_code():
+    x = CASES["two_symbols"]
+    e = (x >> 7) & 0xFF
+    for bad in ({127: 1, 128: 2}, {127: 2, 128: 2}, {127: 17, 128: 1}, {127: 1}):
+        ln = np.zeros(256, np.uint8)
+        for k, v in bad.items():
+            ln[k] = v
+        with pytest.raises(L.Ecf8Error):
+            L.bf16_encode(x, lengths=ln)
+    ln = np.zeros(256, np.uint8)
+    ln[np.unique(e)] = 1  # complete: two 1-bit codes
+    assert np.array_equal(oracle.bf16_decode(L.bf16_encode(x, lengths=ln), x.size), x)
+    one = np.full(100, 0x3F80, np.uint16)
+    ln = np.zeros(256, np.uint8)
+    ln[127] = 4  # a single value may take any length
+    assert np.array_equal(L.bf16_encode(one, lengths=ln), oracle.bf16_encode(one, lengths=ln))
