@@ -97,6 +97,24 @@ struct Batch {
 };
 static_assert(sizeof(Batch) <= 4096, "kernel parameter block");
 
+// Checked builds (-DECF8_CHECKED, libecf8_checked.so) test each index a
+// kernel reads or stores against its buffer; a failed test skips the access
+// and sets ECF8_STATUS_BOUNDS.  Release builds compile the tests away.
+#ifdef ECF8_CHECKED
+__device__ __forceinline__ bool in_bounds(bool ok, int32_t* status) {
+  if (!ok && status) atomicOr(status, ECF8_STATUS_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, int32_t*) { return true; }
+#endif
+
+template <int V>
+__host__ __device__ __forceinline__ uint32_t table_bytes(uint32_t nodes) {
+  const uint32_t entries = (nodes + 1) * 16;
+  return V == kWide ? entries * 8 : V == kNarrow ? entries * 4 : V == kNarrowLane ? entries * 128 : (nodes + 1) * 2048;
+}
+
 struct GroupIn {
   uint32_t w[kWords + 1];
   uint32_t gapw, gapn;
@@ -133,9 +151,10 @@ __device__ __forceinline__ uint32_t pair_bf16(uint32_t p, uint32_t q) {
 // bytes 16u..16u+15.  Whole units take two 16-byte stores; the group's ragged
 // first and last unit store only the weights inside the group, whose
 // positions relative to base are [head, head + count).
-__device__ __forceinline__ void emit_unit(uint16_t* out_base, const uint4* st, uint32_t head, uint32_t count,
-                                          uint32_t u, uint4 kb) {
-  const uint4 ex = st[u];
+template <int V>
+__device__ __forceinline__ void emit_unit(uint16_t* out_base, uint64_t base, uint64_t n, const uint4* st,
+                                          uint32_t head, uint32_t count, uint32_t u, uint4 kb, int32_t* status) {
+  const uint4 ex = in_bounds(4 * u + 4 <= (uint32_t)Cfg<V>::kStageWords, status) ? st[u] : make_uint4(0, 0, 0, 0);
   const uint32_t e4[4] = {ex.x, ex.y, ex.z, ex.w}, k4[4] = {kb.x, kb.y, kb.z, kb.w};
   uint32_t o[8];
 #pragma unroll
@@ -145,13 +164,16 @@ __device__ __forceinline__ void emit_unit(uint16_t* out_base, const uint4* st, u
   }
   const uint32_t r0 = 16 * u;
   if (r0 >= head && r0 + 16 <= head + count) {
-    uint4* dst = reinterpret_cast<uint4*>(out_base + r0);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    if (in_bounds(base + r0 + 16 <= n, status)) {
+      uint4* dst = reinterpret_cast<uint4*>(out_base + r0);
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
   } else {
 #pragma unroll
     for (int k = 0; k < 16; ++k)
-      if (r0 + k >= head && r0 + k < head + count) out_base[r0 + k] = (uint16_t)(o[k >> 1] >> (16 * (k & 1)));
+      if (r0 + k >= head && r0 + k < head + count && in_bounds(base + r0 + k < n, status))
+        out_base[r0 + k] = (uint16_t)(o[k >> 1] >> (16 * (k & 1)));
   }
 }
 
@@ -166,15 +188,17 @@ struct Walker {
   // narrow entry: exponents bits 0-15, node bits 16-23, 8 x count bits 27-31
   static constexpr int kSteps = kNibbles;
   const uint8_t* table;
-  uint32_t lane_term;
+  uint32_t lane_term, limit;
+  int32_t* status;
   uint32_t e = 0;
-  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t lane)
-      : table(t), lane_term(V == kNarrowLane ? lane * 4 : 0) {}
+  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t lane, uint32_t lim, int32_t* st)
+      : table(t), lane_term(V == kNarrowLane ? lane * 4 : 0), limit(lim), status(st) {}
   __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
     const uint32_t nib = nibble_of(sw, j);
     // lane-private: byte (node * 16 + nib) * 128 + lane * 4; shared: (node * 16 + nib) * 4
-    const uint32_t at = V == kNarrowLane ? (((e >> 5) & (0x1Fu << 11)) | (nib << 7) | lane_term)
-                                         : (((e >> 10) & (0xFFu << 6)) | (nib << 2));
+    uint32_t at = V == kNarrowLane ? (((e >> 5) & (0x1Fu << 11)) | (nib << 7) | lane_term)
+                                   : (((e >> 10) & (0xFFu << 6)) | (nib << 2));
+    if (!in_bounds(at + 4 <= limit, status)) at = 0;
     e = *reinterpret_cast<const uint32_t*>(table + at);
     syms = e & 0xFFFFu;
     bits8 = e >> 27;
@@ -186,10 +210,15 @@ template <>
 struct Walker<kWide> {
   static constexpr int kSteps = kNibbles;
   const uint8_t* table;
+  uint32_t limit;
+  int32_t* status;
   uint32_t y = 0;
-  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t) : table(t) {}
+  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t, uint32_t lim, int32_t* st)
+      : table(t), limit(lim), status(st) {}
   __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
-    const uint2 e = *reinterpret_cast<const uint2*>(table + ((y & (0xFFu << 7)) | (nibble_of(sw, j) << 3)));
+    uint32_t at = (y & (0xFFu << 7)) | (nibble_of(sw, j) << 3);
+    if (!in_bounds(at + 8 <= limit, status)) at = 0;
+    const uint2 e = *reinterpret_cast<const uint2*>(table + at);
     y = e.y;
     syms = e.x;
     bits8 = e.y >> 16;
@@ -212,12 +241,17 @@ struct Walker<kByte> {
   // node << 11 | (node & 15) << 3, so one LOP3 gives the next slot's offset
   static constexpr int kSteps = kNibbles / 2;
   const uint8_t* table;
+  uint32_t limit;
+  int32_t* status;
   uint32_t y = 0;
-  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t) : table(t) {}
+  __device__ __forceinline__ Walker(const uint8_t* t, uint32_t, uint32_t lim, int32_t* st)
+      : table(t), limit(lim), status(st) {}
   __device__ __forceinline__ void step(const uint32_t* sw, int j, uint32_t& syms, uint32_t& bits8) {
     const uint32_t b8 = ((sw[j >> 2] >> (24 - 8 * (j & 3))) & 0xFFu) << 3;
     const uint32_t swz8 = b8 ^ ((b8 >> 4) & 0x78u);  // (byte & 0xF0 | (byte ^ byte >> 4) & 15) * 8
-    const uint2 e = *reinterpret_cast<const uint2*>(table + ((y & ((0x1Fu << 11) | (15u << 3))) ^ swz8));
+    uint32_t at = (y & ((0x1Fu << 11) | (15u << 3))) ^ swz8;
+    if (!in_bounds(at + 8 <= limit, status)) at = 0;
+    const uint2 e = *reinterpret_cast<const uint2*>(table + at);
     y = e.y;
     syms = e.x;
     bits8 = e.y >> 24;
@@ -244,7 +278,8 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
 #pragma unroll
   for (int i = 0; i < kKeep; ++i) {
     const uint32_t u = lane + 32 * i;
-    kp[i] = u < units ? __ldg(kept_units + u) : make_uint4(0, 0, 0, 0);
+    kp[i] = u < units && in_bounds((base >> 4) + u < (a.n + 15) / 16, status) ? __ldg(kept_units + u)
+                                                                              : make_uint4(0, 0, 0, 0);
   }
 
   // the lane's bits run from its first code to the next lane's first code or the stream end
@@ -269,7 +304,7 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
   // the lane's capacity, which in a valid stream only the zero padding
   // produces, are counted but not stored)
   uint32_t* priv = wa->priv + lane;
-  Walker<V> walk(table, lane);
+  Walker<V> walk(table, lane, table_bytes<V>(a.nodes), status);
   uint32_t acc = 0, sh = 0, words = 0;
 #pragma unroll
   for (int j = 0; j < Walker<V>::kSteps; ++j) {
@@ -315,7 +350,8 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
   uint32_t* stage = wa->stage;
   const uint32_t q = head + start;
   const uint32_t d0 = q >> 2, dl = cnt ? (q + cnt - 1) >> 2 : 0;
-  if (cnt) {
+  constexpr uint32_t kSW = (uint32_t)C::kStageWords, kPW = (uint32_t)C::kPrivWords;
+  if (cnt && in_bounds(dl < kSW, status)) {
     stage[d0] = 0;
     stage[dl] = 0;
   }
@@ -323,20 +359,20 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
   if (cnt) {
     const uint32_t r = (q & 3) * 8;
     const uint32_t used = (cnt + 3) / 4;
-    if (cnt & 3) priv[32 * (used - 1)] &= (1u << (8 * (cnt & 3))) - 1;
+    if ((cnt & 3) && in_bounds(used - 1 < kPW, status)) priv[32 * (used - 1)] &= (1u << (8 * (cnt & 3))) - 1;
     const uint32_t nwd = dl - d0 + 1;
     uint32_t prev = priv[0];
-    atomicOr(&stage[d0], prev << r);
+    if (in_bounds(d0 < kSW, status)) atomicOr(&stage[d0], prev << r);
     uint32_t j = 1;
 #pragma unroll 4
     for (; j + 1 < nwd; ++j) {
-      const uint32_t cur = priv[32 * j];
-      stage[d0 + j] = __funnelshift_l(prev, cur, r);
+      const uint32_t cur = in_bounds(j < kPW, status) ? priv[32 * j] : 0u;
+      if (in_bounds(d0 + j < kSW, status)) stage[d0 + j] = __funnelshift_l(prev, cur, r);
       prev = cur;
     }
     if (nwd > 1) {
-      const uint32_t cur = j < used ? priv[32 * j] : 0;
-      atomicOr(&stage[d0 + j], __funnelshift_l(prev, cur, r));
+      const uint32_t cur = j < used && in_bounds(j < kPW, status) ? priv[32 * j] : 0;
+      if (in_bounds(d0 + j < kSW, status)) atomicOr(&stage[d0 + j], __funnelshift_l(prev, cur, r));
     }
   }
   __syncwarp();
@@ -347,10 +383,13 @@ __device__ void process_group(const Args& a, uint32_t g, const GroupIn& in, cons
 #pragma unroll
   for (int i = 0; i < kKeep; ++i) {
     const uint32_t u = lane + 32 * i;
-    if (u < units) emit_unit(out_base, st, head, count, u, kp[i]);
+    if (u < units) emit_unit<V>(out_base, base, a.n, st, head, count, u, kp[i], status);
   }
-  for (uint32_t u = lane + 32 * kKeep; u < units; u += 32)
-    emit_unit(out_base, st, head, count, u, __ldg(kept_units + u));
+  for (uint32_t u = lane + 32 * kKeep; u < units; u += 32) {
+    const uint4 kb = in_bounds((base >> 4) + u < (a.n + 15) / 16, status) ? __ldg(kept_units + u)
+                                                                           : make_uint4(0, 0, 0, 0);
+    emit_unit<V>(out_base, base, a.n, st, head, count, u, kb, status);
+  }
   __syncwarp();
 }
 
@@ -440,12 +479,6 @@ __global__ void __launch_bounds__(Cfg<V>::kMaxWarps * 32, 1)
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 uint32_t up16(uint32_t x) { return (x + 15) & ~15u; }
-
-template <int V>
-uint32_t table_bytes(uint32_t nodes) {
-  const uint32_t entries = (nodes + 1) * 16;
-  return V == kWide ? entries * 8 : V == kNarrow ? entries * 4 : V == kNarrowLane ? entries * 128 : (nodes + 1) * 2048;
-}
 
 // One launch over ts[0, count) (count <= ECF8_BF16_BATCH_MAX, every tensor
 // non-empty and holdable by layout V).

@@ -95,3 +95,80 @@ def test_damaged_blobs_never_trip_a_bounds_check(env, seed):
         _, status, intact = _decode(env, [bad])
         assert intact
         assert not status & BOUNDS, status
+
+
+# ---- the BF16 decoder in the checked build ----
+
+def _bf16_decode_checked(env, blob, layout, guard=32):
+    L, torch, so = env
+    so.ecf8_bf16_decode_layout.argtypes = [ctypes.POINTER(L.Bf16Info), ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_int]
+    info = L.bf16_blob_info(blob)
+    d_blob = torch.from_numpy(blob).cuda()
+    d_table = torch.from_numpy(L.bf16_table(info)).cuda()
+    buf = torch.full((info.n + 2 * guard,), 0x3C3C, dtype=torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = so.ecf8_bf16_decode_layout(ctypes.byref(info), d_blob.data_ptr(), d_table.data_ptr(),
+                                    buf.data_ptr() + 2 * guard, info.n, status.data_ptr(),
+                                    torch.cuda.current_stream().cuda_stream, L.BF16_LAYOUTS[layout])
+    assert rc == 0
+    torch.cuda.synchronize()
+    got = buf.cpu().numpy().view(np.uint16)
+    intact = (got[:guard] == 0x3C3C).all() and (got[-guard:] == 0x3C3C).all()
+    return got[guard:-guard], int(status.item()), intact
+
+
+def _bf16_layouts(L, blob):
+    info = L.bf16_blob_info(blob)
+    lens = info.lengths
+    if lens[lens > 0].min() == 1:
+        return ["wide"]
+    return ["wide", "narrow"] + (["narrow_lane", "byte"] if L.bf16_table_nodes(info) + 1 <= 32 else [])
+
+
+def _bf16_inputs():
+    r = np.random.default_rng(17)
+    spec = synth.llama3_8b_layer_bf16().tensors[0]
+    return [spec.generate_bf16(begin=11, count=250_003),                       # byte / narrow_lane / narrow / wide
+            r.integers(0, 1 << 16, 120_001).astype(np.uint16),                # 255 nodes: narrow / wide
+            np.where(r.random(90_001) < 0.95, 0x3F80, 0xC000).astype(np.uint16),  # 1-bit codes: wide
+            spec.generate_bf16(begin=5, count=17)]
+
+
+@pytest.mark.parametrize("k", range(4))
+def test_bf16_valid_blobs_pass_every_check(env, k):
+    L = env[0]
+    x = _bf16_inputs()[k]
+    blob = oracle.bf16_encode(x)
+    for layout in _bf16_layouts(L, blob):
+        got, status, intact = _bf16_decode_checked(env, blob, layout)
+        assert status == 0 and intact, layout
+        assert np.array_equal(got, x), layout
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_bf16_damaged_blobs_never_trip_a_bounds_check(env, seed):
+    L = env[0]
+    r = np.random.default_rng(100 + seed)
+    x = _bf16_inputs()[0]
+    blob = oracle.bf16_encode(x)
+    hd = oracle.bf16_blob_header(blob)
+    damaged = []
+    b = blob.copy()
+    pos = hd["stream_off"] + r.integers(0, hd["code_bits"] // 8, size=150)
+    b[pos] ^= r.integers(1, 256, size=pos.size).astype(np.uint8)
+    damaged.append(b)
+    b = blob.copy()
+    pos = hd["gaps_off"] + r.integers(0, hd["groups_off"] - hd["gaps_off"], size=40)
+    b[pos] = r.integers(0, 256, size=pos.size).astype(np.uint8)
+    damaged.append(b)
+    b = blob.copy()
+    for g in r.integers(1, hd["n_groups"], size=3):
+        b[hd["groups_off"] + 8 * int(g) + int(r.integers(0, 8))] ^= np.uint8(1 << int(r.integers(0, 8)))
+    damaged.append(b)
+    for bad in damaged:
+        for layout in _bf16_layouts(L, blob):
+            _, status, intact = _bf16_decode_checked(env, bad, layout)
+            assert intact, layout
+            assert not status & BOUNDS, (layout, status)
