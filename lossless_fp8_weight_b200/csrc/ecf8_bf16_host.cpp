@@ -305,13 +305,16 @@ struct Tree {
   bool ok = false;
 };
 
-Tree make_tree(const uint8_t* len) {
+// with_order: also list the values in canonical order (the table builder
+// needs it; the node count does not)
+Tree make_tree(const uint8_t* len, bool with_order) {
   Tree t;
   for (int s = 0; s < kSym; ++s)
     if (len[s] && len[s] <= kMaxLen) { ++t.count[len[s]]; ++t.present; t.max_len = std::max<int>(t.max_len, len[s]); }
-  for (int l = 1; l <= kMaxLen; ++l)
-    for (int s = 0; s < kSym; ++s)
-      if (len[s] == l) t.sorted.push_back(s);
+  if (with_order)
+    for (int l = 1; l <= kMaxLen; ++l)
+      for (int s = 0; s < kSym; ++s)
+        if (len[s] == l) t.sorted.push_back(s);
   uint32_t c = 0, b = 0;
   for (int l = 1; l <= kMaxLen; ++l) {
     c = (c + t.count[l - 1]) << 1;
@@ -339,7 +342,7 @@ Tree make_tree(const uint8_t* len) {
 
 extern "C" {
 
-uint32_t ecf8_bf16_table_nodes(const ecf8_bf16_info* info) { return info ? make_tree(info->len).nodes : 0; }
+uint32_t ecf8_bf16_table_nodes(const ecf8_bf16_info* info) { return info ? make_tree(info->len, false).nodes : 0; }
 
 // Entry (node s, nibble v) at index s * 16 + v: x = the exponents whose codes
 // end inside the nibble, 8 bits each, first lowest; y = (next node << 7) |
@@ -349,7 +352,7 @@ uint32_t ecf8_bf16_table_nodes(const ecf8_bf16_info* info) { return info ? make_
 // error node.
 int ecf8_bf16_build_table(const ecf8_bf16_info* info, void* h_table) {
   if (!info || !h_table) return ECF8_ERR_ARG;
-  const Tree T = make_tree(info->len);
+  const Tree T = make_tree(info->len, true);
   const uint32_t err = T.nodes;
   auto step = [&](uint32_t s, uint32_t bit, int* sym) -> uint32_t {
     *sym = -1;
