@@ -35,6 +35,7 @@ import ecf8_synth as synth  # noqa: E402
 
 METRIC = "ECF8 decode GB/s (FP8 out) and % of HBM roofline on 1 B200; compression ratio"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0  # HGX B200 HBM3e specification, for context beside the measured copy peak
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SRC = os.path.join(ROOT, "lossless_fp8_weight_b200", "csrc", "ecf8_decode.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
@@ -687,6 +688,7 @@ def run_bf16(args):
             "ms_per_layer_one_launch_per_tensor": round(ms_separate, 5),
             "roofline": {"bound": "hbm", "achieved": round(alg / ms / 1e6, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(alg / ms / 1e6 / peak, 4),
+                         "frac_of_nominal": round(alg / ms / 1e6 / NOMINAL_HBM_GBS, 4),
                          "algorithmic_bytes": alg, "peak_source": f"{peak_kind} hbm_gbs"},
             "timing": "CUDA graph of the layer's batched launch, replayed; per tensor: graph of 10 launches "
                       "(tensors whose blob + output fit in L2 run L2-warm there)",
@@ -885,7 +887,9 @@ def main():
                        **comp},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": alg_bytes,
+                         "peak_source": f"{peak_kind} hbm_gbs", "nominal_peak": NOMINAL_HBM_GBS,
+                         "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "algorithmic_bytes_per_launch": alg_bytes,
                          "launch_ms": round(per_launch_ms, 5)},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s",
