@@ -162,3 +162,47 @@ def test_round_trip_edge_cases(case):
     }[case]
     blob = oracle.bf16_encode(x)
     assert np.array_equal(oracle.bf16_decode(blob, x.size), x)
+
+
+def _read_bf16_golden():
+    """Key/value lines of tests/golden/bf16_worked_example.txt (comments skipped)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "bf16_worked_example.txt")
+    g = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                k, *v = line.split()
+                g[k] = v
+    return g
+
+
+def test_hand_derived_golden_blob():
+    """The oracle reproduces a blob worked out on paper (the fixture's header
+    gives the derivation): lengths, canonical codes, a code straddling the
+    chunk boundary (gap 1), group offsets, stream words and kept bytes."""
+    g = _read_bf16_golden()
+    x = np.array([int(v, 16) for v in g["weights"]], dtype=np.uint16)
+    C, T = int(g["chunk_bytes"][0]), int(g["group_chunks"][0])
+    blob = oracle.bf16_encode(x, chunk_bytes=C, group_chunks=T)
+    hd = oracle.bf16_blob_header(blob)
+    want_len = np.zeros(256, np.uint8)
+    for kv in g["lengths"]:
+        k, v = kv.split(":")
+        want_len[int(k)] = int(v)
+    assert np.array_equal(hd["lengths"], want_len)
+    codes = oracle.bf16_canonical_codes(want_len)
+    for kv in g["codes"]:
+        k, v = kv.split(":")
+        assert int(codes[int(k)]) == int(v)
+    assert hd["code_bits"] == int(g["code_bits"][0]) and hd["n_groups"] == int(g["n_groups"][0])
+    words = [int(v, 16) for v in g["stream_words"]]
+    assert blob[hd["stream_off"]:hd["stream_off"] + 4 * len(words)].view("<u4").tolist() == words
+    gaps = [int(v, 16) for v in g["gap_words"]]
+    assert blob[hd["gaps_off"]:hd["gaps_off"] + 4 * len(gaps)].view("<u4").tolist() == gaps
+    offs = [int(v) for v in g["group_offsets"]]
+    assert blob[hd["groups_off"]:hd["groups_off"] + 8 * len(offs)].view("<u8").tolist() == offs
+    kept = [int(v, 16) for v in g["kept_bytes"]]
+    assert blob[hd["kept_off"]:hd["kept_off"] + len(kept)].tolist() == kept
+    assert np.array_equal(oracle.bf16_decode(blob, x.size), x)
