@@ -4,18 +4,22 @@
 //
 // The same plan as the ECF8 decoder, with an 8-bit alphabet: one warp per
 // group of 32 chunks of 32 stream bytes; each lane shifts its slice to its
-// first code (the gap), zeroes the bits after its last code and walks 68
-// nibbles through a state machine over the code tree (one entry per (node,
-// nibble): the exponents whose codes end inside the nibble, their count and
-// the next node); zero-padding codes are subtracted by count; a warp scan
+// first code (the gap), zeroes the bits after its last code and walks its
+// 272 bits a nibble (or a byte) at a time through a state machine over the
+// code tree (one entry per (node, nibble or byte): the exponents whose codes
+// end inside it, their count and the next node); zero-padding codes are
+// subtracted by count; a warp scan
 // places each lane's exponents; they are packed a byte each into lane-private
 // shared memory, funnel-shifted into a byte stage, and 16 exponents plus 16
 // kept bytes become 16 BF16 values per lane step.  The group's kept bytes are
 // loaded into registers before its walk, so that their DRAM latency overlaps
 // it; the next group's stream words are loaded before the current group is
-// processed.
+// processed.  One launch covers up to ECF8_BF16_BATCH_MAX tensors of one
+// layout: each persistent CTA takes a contiguous run of their groups and
+// restages its table where the run crosses into the next tensor.
 //
-// Three table layouts, chosen per tensor on the host:
+// Four table layouts; the host picks wide, byte or narrow per tensor (the
+// lane-private one only when asked for):
 //  - wide: when a 1-bit code exists a nibble may end 4 codes; 64-bit entries
 //    {exponents, next node << 7 | 8 count << 16}, as the host builds them;
 //    a group may hold 8192 codes, so 13 warps fit an SM;
