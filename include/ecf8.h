@@ -324,8 +324,9 @@ int ecf8_bf16_code_lengths(const uint16_t* x, size_t n, uint32_t max_len, uint8_
 int ecf8_bf16_encoded_size(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,
                            uint32_t group_chunks, size_t* bytes);
 
-/* Encode n BF16 bit patterns into blob (host, capacity cap); the bytes are
- * those of the oracle's encoder for the same lengths.  ECF8_ERR_CODEBOOK as
+/* Encode n BF16 bit patterns into blob (host, capacity cap; OpenMP threads
+ * over ranges of >= 1M weights); the bytes are those of the oracle's encoder
+ * for the same lengths, whatever the thread count.  ECF8_ERR_CODEBOOK as
  * for ecf8_bf16_encoded_size; ECF8_ERR_CAPACITY if cap is short; *bytes gets
  * the size. */
 int ecf8_bf16_encode(const uint16_t* x, size_t n, const uint8_t len[256], uint32_t chunk_bytes,

@@ -5,6 +5,7 @@
 // and the decode table the GPU kernel walks: one entry per (tree node,
 // 4-bit nibble) giving the exponents whose codes end in the nibble and the
 // node after it.
+#include <omp.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -147,14 +148,98 @@ bool canonical(const uint8_t* len, uint32_t* code) {
   return true;
 }
 
+// Host threads for n weights: ranges of at least 1M weights.
+int parts_for(size_t n) {
+  const size_t per = (size_t)1 << 20;
+  const size_t want = (n + per - 1) / per;
+  const size_t t = (size_t)std::max(1, omp_get_max_threads());
+  return (int)std::max<size_t>(1, std::min(t, want));
+}
+
+// Code bits of weights [i0, i1); false when an exponent there has no code.
+bool range_bits(const uint16_t* x, size_t i0, size_t i1, const uint8_t* len, uint64_t* bits) {
+  uint64_t b = 0;
+  bool ok = true;
+  for (size_t i = i0; i < i1; ++i) {
+    const uint8_t l = len[(x[i] >> 7) & 0xFF];
+    ok &= l != 0;
+    b += l;
+  }
+  *bits = b;
+  return ok;
+}
+
+// Bits of each of `parts` equal weight ranges, as a prefix sum (range_bit[p]
+// is where range p's first code starts); false when an exponent has no code.
+bool prefix_bits(const uint16_t* x, size_t n, const uint8_t* len, int parts, std::vector<uint64_t>* range_bit) {
+  range_bit->assign(parts + 1, 0);
+  std::vector<uint64_t> bits(parts, 0);
+  std::vector<char> ok(parts, 1);
+#pragma omp parallel for num_threads(parts) schedule(static, 1)
+  for (int p = 0; p < parts; ++p)
+    ok[p] = range_bits(x, n * (size_t)p / parts, n * (size_t)(p + 1) / parts, len, &bits[p]) ? 1 : 0;
+  for (int p = 0; p < parts; ++p) {
+    if (!ok[p]) return false;
+    (*range_bit)[p + 1] = (*range_bit)[p] + bits[p];
+  }
+  return true;
+}
+
+// Codes of weights [i0, i1) into the stream from bit bit0, with the gap and
+// group offset of every chunk that starts in [bit0, bit1) (bit1: where code
+// i1 starts, or the stream end).  Words shared with the neighbouring ranges
+// are OR-ed atomically into a zeroed stream.
+void pack(const uint16_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t bit1, const uint8_t* len,
+          const uint32_t* code, uint64_t chunk_bits, uint32_t T, uint64_t chunks, uint32_t* stream, uint32_t* gaps,
+          uint64_t* offs) {
+  uint64_t chunk = (bit0 + chunk_bits - 1) / chunk_bits;  // the first chunk starting at or after bit0
+  uint64_t boundary = chunk * chunk_bits;
+  auto put_gap = [&](uint64_t c, uint64_t gap, uint64_t first_code) {
+    __atomic_fetch_or(&gaps[c / 8], (uint32_t)gap << (4 * (c % 8)), __ATOMIC_RELAXED);
+    if (c % T == 0) offs[c / T] = first_code;
+  };
+  const uint64_t first_word = bit0 / 32;
+  uint64_t word = first_word, pos = bit0, acc = 0;
+  uint32_t nacc = (uint32_t)(bit0 % 32);  // the previous range's bits of the first word stay zero here
+  for (size_t i = i0; i < i1; ++i) {
+    while (chunk < chunks && boundary <= pos) {  // at most once: a code is <= 16 bits, a chunk >= 32
+      put_gap(chunk, pos - boundary, i);
+      ++chunk;
+      boundary += chunk_bits;
+    }
+    const uint32_t e = (x[i] >> 7) & 0xFF;
+    acc = (acc << len[e]) | code[e];
+    nacc += len[e];
+    pos += len[e];
+    if (nacc >= 32) {
+      nacc -= 32;
+      const uint32_t v = (uint32_t)(acc >> nacc);
+      if (word == first_word)
+        __atomic_fetch_or(&stream[word], v, __ATOMIC_RELAXED);
+      else
+        stream[word] = v;
+      ++word;
+    }
+  }
+  if (nacc) __atomic_fetch_or(&stream[word], (uint32_t)(acc << (32 - nacc)), __ATOMIC_RELAXED);
+  for (; chunk < chunks && boundary < bit1; ++chunk, boundary += chunk_bits) put_gap(chunk, bit1 - boundary, i1);
+}
+
 }  // namespace
 
 extern "C" {
 
 int ecf8_bf16_code_lengths(const uint16_t* x, size_t n, uint32_t max_len, uint8_t len[256]) {
   if (!len || (!x && n) || max_len < 1 || max_len > kMaxLen) return ECF8_ERR_ARG;
-  std::vector<uint64_t> h(kSym, 0);
-  for (size_t i = 0; i < n; ++i) ++h[(x[i] >> 7) & 0xFF];
+  const int parts = parts_for(n);
+  std::vector<uint64_t> ph((size_t)parts * kSym, 0), h(kSym, 0);
+#pragma omp parallel for num_threads(parts) schedule(static, 1)
+  for (int p = 0; p < parts; ++p) {
+    uint64_t* hp = ph.data() + (size_t)p * kSym;
+    for (size_t i = n * (size_t)p / parts, e = n * (size_t)(p + 1) / parts; i < e; ++i) ++hp[(x[i] >> 7) & 0xFF];
+  }
+  for (int p = 0; p < parts; ++p)
+    for (int v = 0; v < kSym; ++v) h[v] += ph[(size_t)p * kSym + v];
   huffman(h.data(), len);
   int deepest = 0;
   for (int s = 0; s < kSym; ++s) deepest = std::max<int>(deepest, len[s]);
@@ -166,14 +251,10 @@ int ecf8_bf16_encoded_size(const uint16_t* x, size_t n, const uint8_t len[256], 
                            uint32_t group_chunks, size_t* bytes) {
   if (!len || !bytes || (!x && n)) return ECF8_ERR_ARG;
   if (!valid_lengths(len)) return ECF8_ERR_CODEBOOK;
-  uint64_t bits = 0;
-  for (size_t i = 0; i < n; ++i) {
-    const uint8_t l = len[(x[i] >> 7) & 0xFF];
-    if (!l) return ECF8_ERR_CODEBOOK;
-    bits += l;
-  }
+  std::vector<uint64_t> range_bit;
+  if (!prefix_bits(x, n, len, parts_for(n), &range_bit)) return ECF8_ERR_CODEBOOK;
   Layout L;
-  if (!layout(n, bits, chunk_bytes, group_chunks, &L)) return ECF8_ERR_ARG;
+  if (!layout(n, range_bit.back(), chunk_bytes, group_chunks, &L)) return ECF8_ERR_ARG;
   *bytes = L.total;
   return ECF8_OK;
 }
@@ -183,14 +264,12 @@ int ecf8_bf16_encode(const uint16_t* x, size_t n, const uint8_t len[256], uint32
   if (!len || !blob_v || !bytes || (!x && n)) return ECF8_ERR_ARG;
   uint32_t code[kSym];
   if (!valid_lengths(len) || !canonical(len, code)) return ECF8_ERR_CODEBOOK;
-  uint64_t bits = 0;
   int max_len = 0;
   for (int s = 0; s < kSym; ++s) max_len = std::max<int>(max_len, len[s]);
-  for (size_t i = 0; i < n; ++i) {
-    const uint8_t l = len[(x[i] >> 7) & 0xFF];
-    if (!l) return ECF8_ERR_CODEBOOK;
-    bits += l;
-  }
+  const int parts = parts_for(n);
+  std::vector<uint64_t> range_bit;
+  if (!prefix_bits(x, n, len, parts, &range_bit)) return ECF8_ERR_CODEBOOK;
+  const uint64_t bits = range_bit.back();
   Layout L;
   if (!layout(n, bits, chunk_bytes, group_chunks, &L)) return ECF8_ERR_ARG;
   if (cap < L.total) return ECF8_ERR_CAPACITY;
@@ -215,30 +294,18 @@ int ecf8_bf16_encode(const uint16_t* x, size_t n, const uint8_t len[256], uint32
   uint32_t* gaps = reinterpret_cast<uint32_t*>(b + L.gaps_off);
   uint64_t* offs = reinterpret_cast<uint64_t*>(b + L.groups_off);
   const uint64_t chunk_bits = 8ull * chunk_bytes, chunks = L.groups * group_chunks;
-  uint64_t next_chunk = 0, pos = 0, acc = 0, word = 0;
-  uint32_t nacc = 0;
-  for (size_t i = 0; i <= n; ++i) {
-    while (next_chunk < chunks && next_chunk * chunk_bits <= pos) {  // at most one: codes <= 16 bits
-      const uint64_t gap = pos - next_chunk * chunk_bits;
-      gaps[next_chunk / 8] |= (uint32_t)gap << (4 * (next_chunk % 8));
-      if (next_chunk % group_chunks == 0) offs[next_chunk / group_chunks] = i;
-      ++next_chunk;
-    }
-    if (i == n) break;
-    const uint32_t e = (x[i] >> 7) & 0xFF;
-    acc = (acc << len[e]) | code[e];
-    nacc += len[e];
-    pos += len[e];
-    if (nacc >= 32) {
-      nacc -= 32;
-      stream[word++] = (uint32_t)(acc >> nacc);
-    }
-  }
-  if (nacc) stream[word] = (uint32_t)(acc << (32 - nacc));
-  for (; next_chunk < chunks; ++next_chunk)
-    if (next_chunk % group_chunks == 0) offs[next_chunk / group_chunks] = n;
+#pragma omp parallel for num_threads(parts) schedule(static, 1)
+  for (int p = 0; p < parts; ++p)
+    pack(x, n * (size_t)p / parts, n * (size_t)(p + 1) / parts, range_bit[p], range_bit[p + 1], len, code,
+         chunk_bits, group_chunks, chunks, stream, gaps, offs);
+  // a chunk that starts at or after the stream end: gap 0, its group begins at n
+  for (uint64_t c = (bits + chunk_bits - 1) / chunk_bits; c < chunks; ++c)
+    if (c % group_chunks == 0) offs[c / group_chunks] = n;
   offs[L.groups] = n;
-  for (size_t i = 0; i < n; ++i) b[L.kept_off + i] = (uint8_t)(((x[i] >> 15) << 7) | (x[i] & 0x7F));
+  uint8_t* kept = b + L.kept_off;
+  const long long nn = (long long)n;
+#pragma omp parallel for num_threads(parts) schedule(static)
+  for (long long i = 0; i < nn; ++i) kept[i] = (uint8_t)(((x[i] >> 15) << 7) | (x[i] & 0x7F));
   *bytes = L.total;
   return ECF8_OK;
 }

@@ -289,3 +289,17 @@ def test_encoder_refuses_lengths_that_are_not_a_complete_code():
     ln = np.zeros(256, np.uint8)
     ln[127] = 4  # a single value may take any length
     assert np.array_equal(L.bf16_encode(one, lengths=ln), oracle.bf16_encode(one, lengths=ln))
+
+
+@pytest.mark.parametrize("C,T", [(32, 32), (4, 1), (12, 5)])
+def test_threaded_encoder_matches_the_serial_oracle(C, T):
+    """Over 1M weights a thread the library packs ranges concurrently (shared
+    boundary words OR-ed, gaps and offsets per range); the bytes must not
+    depend on that split."""
+    import ecf8_synth as synth
+    x = synth.llama3_8b_layer_bf16().tensors[1].generate_bf16(begin=99, count=3_300_017)
+    x[::4099] ^= 0x4000  # a wider exponent spread
+    ln = L.bf16_code_lengths(x)
+    assert np.array_equal(ln, oracle.bf16_blob_header(oracle.bf16_encode(x[:1000], lengths=ln))["lengths"])
+    assert np.array_equal(L.bf16_encode(x, lengths=ln, chunk_bytes=C, group_chunks=T),
+                          oracle.bf16_encode(x, lengths=ln, chunk_bytes=C, group_chunks=T))
