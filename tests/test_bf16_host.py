@@ -303,3 +303,56 @@ def test_threaded_encoder_matches_the_serial_oracle(C, T):
     assert np.array_equal(ln, oracle.bf16_blob_header(oracle.bf16_encode(x[:1000], lengths=ln))["lengths"])
     assert np.array_equal(L.bf16_encode(x, lengths=ln, chunk_bytes=C, group_chunks=T),
                           oracle.bf16_encode(x, lengths=ln, chunk_bytes=C, group_chunks=T))
+
+
+FAKE = 1 << 20  # a 16-byte-aligned address that is never dereferenced
+
+
+def test_argument_errors_are_returned_before_any_device_work():
+    """Every error path of the BF16 entry points returns before a CUDA call,
+    so it can be exercised without a GPU."""
+    import ctypes
+    lib = L._lib
+    ARG, CODEBOOK, CAPACITY, ALIGN, UNSUPPORTED = -1, -4, -3, -5, -6
+    x = CASES["normal"]
+    ln = L.bf16_code_lengths(x)
+    size = ctypes.c_size_t(0)
+    assert lib.ecf8_bf16_code_lengths(x.ctypes.data, x.size, 16, None) == ARG
+    assert lib.ecf8_bf16_code_lengths(x.ctypes.data, x.size, 0, ln.ctypes.data) == ARG
+    assert lib.ecf8_bf16_code_lengths(x.ctypes.data, x.size, 17, ln.ctypes.data) == ARG
+    assert lib.ecf8_bf16_encoded_size(x.ctypes.data, x.size, ln.ctypes.data, 6, 32, ctypes.byref(size)) == ARG
+    assert lib.ecf8_bf16_encoded_size(x.ctypes.data, x.size, ln.ctypes.data, 32, 0, ctypes.byref(size)) == ARG
+    assert lib.ecf8_bf16_encoded_size(x.ctypes.data, x.size, ln.ctypes.data, 32, 32, None) == ARG
+    assert lib.ecf8_bf16_encoded_size(x.ctypes.data, x.size, ln.ctypes.data, 32, 32, ctypes.byref(size)) == 0
+    small = np.zeros(size.value - 1, np.uint8)
+    got = ctypes.c_size_t(0)
+    assert lib.ecf8_bf16_encode(x.ctypes.data, x.size, ln.ctypes.data, 32, 32, small.ctypes.data, small.size,
+                                ctypes.byref(got)) == CAPACITY
+    assert lib.ecf8_bf16_blob_info(None, 0, None) == ARG
+    assert lib.ecf8_bf16_build_table(None, FAKE) == ARG
+    assert lib.ecf8_bf16_table_nodes(None) == 0
+    assert lib.ecf8_bf16_auto_layout(None) == ARG
+
+    blob = L.bf16_encode(x)
+    info = L.bf16_blob_info(blob)
+    dec = lib.ecf8_bf16_decode_layout
+    ref = ctypes.byref(info)
+    assert dec(ref, FAKE, FAKE, FAKE, info.n + 1, None, None, -1) == ARG          # n differs from the header
+    assert dec(ref, FAKE, FAKE, FAKE, info.n, None, None, 7) == ARG               # no such layout
+    assert dec(ref, None, FAKE, FAKE, info.n, None, None, -1) == ARG              # null blob
+    assert dec(ref, FAKE + 4, FAKE, FAKE, info.n, None, None, -1) == ALIGN        # unaligned blob
+    assert dec(ref, FAKE, FAKE, FAKE + 2, info.n, None, None, -1) == ALIGN        # unaligned output
+    wide_only = L.bf16_blob_info(L.bf16_encode(CASES["two_symbols"]))
+    assert dec(ctypes.byref(wide_only), FAKE, FAKE, FAKE, wide_only.n, None, None, 3) == UNSUPPORTED
+    other = L.bf16_blob_info(L.bf16_encode(x, chunk_bytes=16, group_chunks=8))
+    assert dec(ctypes.byref(other), FAKE, FAKE, FAKE, other.n, None, None, -1) == UNSUPPORTED
+    empty = L.bf16_blob_info(L.bf16_encode(np.zeros(0, np.uint16)))
+    assert dec(ctypes.byref(empty), None, None, None, 0, None, None, -1) == 0    # nothing to do
+
+    T = L.Bf16Tensor
+    assert lib.ecf8_bf16_decode_batched(None, -1, None, None) == ARG
+    assert lib.ecf8_bf16_decode_batched(None, 0, None, None) == 0
+    arr = (T * 2)(T(ctypes.pointer(info), FAKE, FAKE, FAKE), T(ctypes.pointer(other), FAKE, FAKE, FAKE))
+    assert lib.ecf8_bf16_decode_batched(arr, 2, None, None) == UNSUPPORTED    # checked before anything runs
+    arr = (T * 1)(T(None, FAKE, FAKE, FAKE))
+    assert lib.ecf8_bf16_decode_batched(arr, 1, None, None) == ARG
