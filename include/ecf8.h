@@ -12,41 +12,46 @@
  * Conventions for every call:
  *  - Return value: ECF8_OK (0) or a negative ECF8_ERR_* code; ecf8_strerror
  *    names it.  No call throws, aborts or prints.
- *  - The caller owns every buffer, host and device.  The library keeps no
- *    state between calls except per-device kernel attributes set once, and a
- *    launch counter; it allocates no device memory.
+ *  - The caller owns every buffer, host and device.  Between calls the
+ *    library keeps per-device kernel attributes (set once), a launch counter,
+ *    and one device table of its own: ECF8_NOALLOC_MAX_TENSORS descriptors of
+ *    96 bytes on every GPU that loads the library, used only by
+ *    ecf8_decode_batched_noalloc, overwritten by each such call and held until
+ *    the process exits.  No call allocates device memory.
  *  - "host" pointers are ordinary CPU memory; "device" pointers are CUDA
  *    global memory of the current device and must be 16-byte aligned.
  *  - Decode calls are asynchronous on the given stream.  Argument and header
  *    errors are returned before anything is enqueued.  Corrupt data found by
  *    the kernel is reported by OR-ing ECF8_STATUS_* bits into *d_status
  *    (device int32, nullable), which the caller reads after synchronising.
- *    The kernels never write outside [d_out, d_out + n) and never wait.
+ *    The kernels never read outside [d_blob, d_blob + blob_size), never write
+ *    outside [d_out, d_out + n) and never wait.
  *
- * Blob layout (version 1, all fields little-endian; the on-disk and in-HBM
+ * Blob layout (version 2, all fields little-endian; the on-disk and in-HBM
  * form of one compressed tensor):
  *   header, 128 bytes:
- *     0 u32 magic 0x38464345 ("ECF8")   4 u32 version = 1
+ *     0 u32 magic 0x38464345 ("ECF8")   4 u32 version = 2
  *     8 u64 n (weights)                16 u64 code_bits (stream length in bits)
  *    24 u32 chunk_bytes C              28 u32 group_chunks T
- *    32 u32 n_groups G                 36 u32 lut_bits = 12
+ *    32 u32 n_groups G                 36 u32 reserved = 0
  *    40 u32 max code length            44 u32 header bytes = 128
- *    48 u64 offset of decode table     56 u64 offset of gaps
+ *    48 u64 reserved = 0               56 u64 offset of gaps
  *    64 u64 offset of group offsets    72 u64 offset of code stream
  *    80 u64 offset of nibbles          88 u64 blob bytes
  *    96 u8[16] code length per exponent value (0 = absent)   112 u8[16] zero
  *   sections, each at a multiple of 256 bytes, in this order:
- *     decode table  4096 u32 (absent when n = 0).  Entry for a 12-bit window:
- *                   bits 0-3 bits used, 4-6 codes (0..6), 8+4j exponent j,
- *                   the greedy decode of the codes lying wholly in the window.
  *     gaps          4 bits per chunk, chunk c in bits 4(c%8) of u32 word c/8;
  *                   offset of the first code start at or after the chunk start
  *                   (the stream end counts as a start), 0 past the end.
  *     group offsets G+1 u64: number of codes starting before bit 8*C*T*g.
  *     code stream   G*T*C bytes + 16 zero bytes; u32 words, stream bit i is
  *                   bit 31-(i%32) of word i/32.
- *     nibbles       ceil(n/32)*16 bytes; weight i's (sign<<3 | mantissa) in
- *                   byte 4(i/8)+(i%4), low half if i%8 < 4 else high half.
+ *     nibbles       ceil(n/32)*16 bytes, 8 weights per u32 word w: byte k
+ *                   (k = 0..3) holds weight 8w+k's sign in bit 7 and mantissa
+ *                   in bits 0-2, weight 8w+4+k's mantissa in bits 4-6, and in
+ *                   bit 3 the sign of weight 8w+4+((k+3)%4).
+ * The 16 code lengths are the whole codebook: the canonical code follows from
+ * them, and the decoder builds its tables from them.
  */
 #ifndef ECF8_H_
 #define ECF8_H_
@@ -60,7 +65,7 @@
 extern "C" {
 #endif
 
-#define ECF8_ABI_VERSION 1
+#define ECF8_ABI_VERSION 2
 
 /* return codes */
 #define ECF8_OK 0
@@ -73,6 +78,7 @@ extern "C" {
 #define ECF8_ERR_CUDA (-7)        /* a CUDA runtime call failed */
 #define ECF8_ERR_WORKSPACE (-8)   /* workspace null or too small */
 #define ECF8_ERR_TOO_MANY (-9)    /* more tensors than ecf8_decode_batched_noalloc holds */
+#define ECF8_ERR_CAPTURE (-10)    /* a call that copies from host memory was made while its stream captures */
 
 /* bits OR-ed into *d_status by the decode kernels */
 #define ECF8_STATUS_COUNT_MISMATCH 1 /* codes decoded in a group != its offset delta */
@@ -94,11 +100,10 @@ typedef struct ecf8_info {
   uint64_t n;
   uint64_t code_bits;
   uint64_t blob_bytes;
-  uint64_t lut_off, gaps_off, groups_off, stream_off, nibbles_off;
+  uint64_t gaps_off, groups_off, stream_off, nibbles_off;
   uint32_t chunk_bytes;
   uint32_t group_chunks;
   uint32_t n_groups;
-  uint32_t lut_bits;
   uint32_t max_len;
   uint8_t len[16];
 } ecf8_info;
@@ -106,7 +111,8 @@ typedef struct ecf8_info {
 /* One tensor of a batched decode. */
 typedef struct ecf8_tensor {
   const ecf8_info* info; /* host */
-  const void* d_blob;    /* device, 16-byte aligned, info->blob_bytes long */
+  const void* d_blob;    /* device, 16-byte aligned */
+  size_t blob_size;      /* bytes readable at d_blob; at least info->blob_bytes */
   uint8_t* d_out;        /* device, 16-byte aligned, info->n bytes */
 } ecf8_tensor;
 
@@ -121,28 +127,51 @@ int ecf8_histogram(const uint8_t* fp8, size_t n, uint64_t hist[16]);
  * code.  ECF8_ERR_CODEBOOK when 2^max_len < number of present values. */
 int ecf8_build_codebook(const uint64_t hist[16], uint32_t max_len, ecf8_codebook* out);
 
-/* Exact blob size for n weights with histogram hist under cb.  host. */
+/* Exact blob size for n weights with histogram hist under cb (the
+ * compressed size the ECF8 walkthrough §3.1.1 reports as the memory saving:
+ * code bits from the histogram, plus the per-chunk and per-group metadata of
+ * §3.2.1 and the raw sign/mantissa nibbles).  host.  ECF8_ERR_CODEBOOK if an
+ * exponent in hist has no code; ECF8_ERR_ARG on a bad layout or when the
+ * histogram does not sum to n. */
 int ecf8_encoded_size(const uint64_t hist[16], size_t n, const ecf8_codebook* cb,
                       uint32_t chunk_bytes, uint32_t group_chunks, size_t* out_bytes);
 
-/* Encode n E4M3 bytes into blob (host, capacity cap).  chunk_bytes is the
- * stream slice of one decoder thread (multiple of 4), group_chunks the chunks
- * that share one group offset.  ECF8_ERR_CODEBOOK if a present exponent has
- * no code; ECF8_ERR_CAPACITY if cap is short.  *blob_bytes gets the size. */
+/* An upper bound on the blob size of ANY n weights under any code of at most
+ * 16 bits, with this layout, that needs no histogram (for sizing a buffer
+ * before the weights are seen).  0 for an invalid layout or an n so large the
+ * bound overflows. */
+size_t ecf8_encoded_size_bound(size_t n, uint32_t chunk_bytes, uint32_t group_chunks);
+
+/* Encode n E4M3 bytes into blob (host, capacity cap): the ECF8 walkthrough
+ * §3.1.1 steps (exponent field coded with cb, sign and mantissa kept raw)
+ * and the per-thread metadata of §3.2.1, in the version-2 layout above.
+ * chunk_bytes is the stream slice of one decoder thread (multiple of 4),
+ * group_chunks the chunks that share one group offset.  ECF8_ERR_CODEBOOK if
+ * a present exponent has no code or cb's codes are not the canonical code of
+ * its lengths; ECF8_ERR_CAPACITY if cap is short.  *blob_bytes gets the size.
+ * Multi-threaded over ranges of >= 1M weights; the bytes do not depend on the
+ * thread count. */
 int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t chunk_bytes,
                 uint32_t group_chunks, void* blob, size_t cap, size_t* blob_bytes);
 
-/* Parse and check a host copy of a blob: magic, version, layout, lengths
- * (Kraft sum <= 1) and the decode table against the lengths. */
+/* Parse and check a host copy of a blob (the metadata a decoder of the ECF8
+ * walkthrough §3.2.1 is given beside the bitstream): magic, version, the
+ * section layout against n, code_bits, C and T, and the code lengths (a
+ * prefix code of at most 16 bits, Kraft sum <= 1).  Reads only the 128-byte
+ * header; size is the bytes available at blob.  ECF8_ERR_FORMAT,
+ * ECF8_ERR_CODEBOOK. */
 int ecf8_blob_info(const void* blob, size_t size, ecf8_info* out);
 
 /* 1 if the GPU kernels implement (chunk_bytes, group_chunks), else 0. */
 int ecf8_layout_supported(uint32_t chunk_bytes, uint32_t group_chunks);
 
-/* Decode one tensor on the GPU (§3.2.1): d_blob (device copy of the blob
- * described by info) -> d_out, n must equal info->n.  One kernel launch on
- * stream s; no launch when n = 0. */
-int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_t n,
+/* Decode one tensor on the GPU (ECF8 walkthrough §3.2.1, decode_kernel over
+ * the bitstream and its metadata): d_blob (device copy of the blob described
+ * by info, blob_size bytes readable) -> d_out (n bytes).  n must equal
+ * info->n and blob_size must be at least info->blob_bytes (ECF8_ERR_ARG
+ * otherwise, before anything is enqueued).  One kernel launch on stream s; no
+ * launch when n = 0. */
+int ecf8_decode(const ecf8_info* info, const void* d_blob, size_t blob_size, uint8_t* d_out, size_t n,
                 int32_t* d_status, cudaStream_t s);
 
 /* Batches of at most this many tensors need no workspace. */
@@ -153,12 +182,16 @@ int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_
 size_t ecf8_batched_workspace_size(int count);
 
 /* Decode count tensors in ONE kernel launch (batching across tensors as in
- * the DFloat11 article's block-level batching, "Transformer块级批处理").  All
- * tensors must share chunk_bytes and group_chunks.  Up to
- * ECF8_BATCH_INLINE_MAX tensors travel in the launch's parameter block and
- * d_workspace may be NULL.  Larger batches copy a descriptor table host->device
- * into d_workspace (device, 16-byte aligned) on stream s before the launch;
- * the workspace must not be touched by other streams until the decode ends. */
+ * the DFloat11 article's block-level batching, §3.3).  All tensors must share
+ * chunk_bytes and group_chunks; each tensor's blob_size must cover its
+ * info->blob_bytes (ECF8_ERR_ARG).  Up to ECF8_BATCH_INLINE_MAX tensors travel
+ * in the launch's parameter block and d_workspace may be NULL.  Larger batches
+ * copy a descriptor table from host memory into d_workspace (device, 16-byte
+ * aligned) on stream s before the launch; the workspace must not be touched by
+ * other streams until the decode ends.  That copy reads a temporary host
+ * array, so such a call returns ECF8_ERR_CAPTURE, enqueueing nothing, while s
+ * is capturing a CUDA graph; batches of up to ECF8_BATCH_INLINE_MAX tensors
+ * copy nothing from the host. */
 int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace, size_t workspace_bytes,
                         int32_t* d_status, cudaStream_t s);
 
@@ -174,8 +207,8 @@ int ecf8_decode_batched(const ecf8_tensor* tensors, int count, void* d_workspace
  *
  * The descriptor table that ecf8_decode_batched copies into the caller's
  * workspace goes instead into one table in device memory that the library
- * itself holds: ECF8_NOALLOC_MAX_TENSORS entries of 96 bytes (96 KB) on every
- * GPU that loads the library, kept until the process exits.  The caller
+ * itself holds: ECF8_NOALLOC_MAX_TENSORS entries of 96 bytes (96 KB) on
+ * every GPU that loads the library, kept until the process exits.  The caller
  * still provides every blob and output buffer.  The call makes no cudaMalloc,
  * cudaFree or other allocating call.
  *  - The first call on a device resolves that table's device address (and
@@ -245,6 +278,7 @@ int ecf8_decode_batched_ctas(const ecf8_tensor* tensors, int count, void* d_work
 typedef struct ecf8_layer_tensor {
   const ecf8_info* info; /* host; copied at create time */
   const void* d_blob;    /* device, 16-byte aligned, stays valid while the pipeline lives */
+  size_t blob_size;      /* bytes readable at d_blob; at least info->blob_bytes */
   size_t out_offset;     /* byte offset of its FP8 output within a slot; multiple of 16 (of 32 for
                             the fastest stores); out_offset + info->n <= slot_bytes */
 } ecf8_layer_tensor;
@@ -390,7 +424,10 @@ typedef struct ecf8_bf16_tensor {
 /* Decode count BF16 blobs: one launch per table layout present (AUTO per
  * tensor) and per ECF8_BF16_BATCH_MAX tensors, each CTA over a contiguous
  * run of the tensors' groups.  Every tensor is checked before anything is
- * enqueued (errors as ecf8_bf16_decode); empty tensors are skipped. */
+ * enqueued (argument errors as ecf8_bf16_decode); empty tensors are skipped.
+ * A CUDA error from a launch (ECF8_ERR_CUDA) can come after earlier launches
+ * of the same call were enqueued: some outputs may then be decoded and others
+ * not. */
 int ecf8_bf16_decode_batched(const ecf8_bf16_tensor* tensors, int count, int32_t* d_status, cudaStream_t stream);
 
 /* The layout ecf8_bf16_decode picks for info's code (>= 0), or an error. */

@@ -40,7 +40,7 @@ _lib = ctypes.CDLL(_SO)
 
 OK = 0
 ERRORS = {-1: "ARG", -2: "FORMAT", -3: "CAPACITY", -4: "CODEBOOK", -5: "ALIGN", -6: "UNSUPPORTED", -7: "CUDA",
-          -8: "WORKSPACE", -9: "TOO_MANY"}
+          -8: "WORKSPACE", -9: "TOO_MANY", -10: "CAPTURE"}
 STATUS_COUNT_MISMATCH = 1
 STATUS_BAD_CODE = 2
 STATUS_BAD_OFFSETS = 4
@@ -61,10 +61,10 @@ class Codebook(ctypes.Structure):
 
 class Info(ctypes.Structure):
     _fields_ = [("n", ctypes.c_uint64), ("code_bits", ctypes.c_uint64), ("blob_bytes", ctypes.c_uint64),
-                ("lut_off", ctypes.c_uint64), ("gaps_off", ctypes.c_uint64), ("groups_off", ctypes.c_uint64),
+                ("gaps_off", ctypes.c_uint64), ("groups_off", ctypes.c_uint64),
                 ("stream_off", ctypes.c_uint64), ("nibbles_off", ctypes.c_uint64),
                 ("chunk_bytes", ctypes.c_uint32), ("group_chunks", ctypes.c_uint32), ("n_groups", ctypes.c_uint32),
-                ("lut_bits", ctypes.c_uint32), ("max_len", ctypes.c_uint32), ("len", ctypes.c_uint8 * 16)]
+                ("max_len", ctypes.c_uint32), ("len", ctypes.c_uint8 * 16)]
 
     @property
     def lengths(self) -> np.ndarray:
@@ -76,17 +76,20 @@ class Info(ctypes.Structure):
 
 
 class Tensor(ctypes.Structure):
-    _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("d_out", ctypes.c_void_p)]
+    _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("blob_size", ctypes.c_size_t),
+                ("d_out", ctypes.c_void_p)]
 
 
 _p, _sz, _u32, _i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_int
 _lib.ecf8_histogram.argtypes = [_p, _sz, _p]
 _lib.ecf8_build_codebook.argtypes = [_p, _u32, ctypes.POINTER(Codebook)]
 _lib.ecf8_encoded_size.argtypes = [_p, _sz, ctypes.POINTER(Codebook), _u32, _u32, ctypes.POINTER(_sz)]
+_lib.ecf8_encoded_size_bound.argtypes = [_sz, _u32, _u32]
+_lib.ecf8_encoded_size_bound.restype = _sz
 _lib.ecf8_encode.argtypes = [_p, _sz, ctypes.POINTER(Codebook), _u32, _u32, _p, _sz, ctypes.POINTER(_sz)]
 _lib.ecf8_blob_info.argtypes = [_p, _sz, ctypes.POINTER(Info)]
 _lib.ecf8_layout_supported.argtypes = [_u32, _u32]
-_lib.ecf8_decode.argtypes = [ctypes.POINTER(Info), _p, _p, _sz, _p, _p]
+_lib.ecf8_decode.argtypes = [ctypes.POINTER(Info), _p, _sz, _p, _sz, _p, _p]
 _lib.ecf8_batched_workspace_size.argtypes = [_i32]
 _lib.ecf8_batched_workspace_size.restype = _sz
 _lib.ecf8_decode_batched.argtypes = [ctypes.POINTER(Tensor), _i32, _p, _sz, _p, _p]
@@ -139,7 +142,8 @@ _lib.ecf8_bf16_decode_batched.argtypes = [ctypes.POINTER(Bf16Tensor), _i32, _p, 
 
 
 class LayerTensor(ctypes.Structure):
-    _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("out_offset", ctypes.c_size_t)]
+    _fields_ = [("info", ctypes.POINTER(Info)), ("d_blob", ctypes.c_void_p), ("blob_size", ctypes.c_size_t),
+                ("out_offset", ctypes.c_size_t)]
 
 
 class Layer(ctypes.Structure):
@@ -251,6 +255,11 @@ def encode_device(d_fp8, codebook: Optional[Codebook] = None, chunk_bytes: int =
     return blob
 
 
+def encoded_size_bound(n: int, chunk_bytes: int = DEFAULT_CHUNK_BYTES, group_chunks: int = DEFAULT_GROUP_CHUNKS) -> int:
+    """Blob bytes that suffice for any n weights in this layout (no histogram needed)."""
+    return int(_lib.ecf8_encoded_size_bound(n, chunk_bytes, group_chunks))
+
+
 def blob_info(blob) -> Info:
     b = _host_u8(blob)
     info = Info()
@@ -270,6 +279,13 @@ def _ptr(t) -> int:
     return int(t.data_ptr())
 
 
+def _nbytes(t, default: int) -> int:
+    """Bytes of a torch tensor argument; a raw pointer is taken to hold `default`."""
+    if t is None or isinstance(t, int):
+        return int(default)
+    return int(t.numel() * t.element_size())
+
+
 def _stream(stream) -> int:
     if stream is None:
         import torch
@@ -279,10 +295,13 @@ def _stream(stream) -> int:
     return int(stream.cuda_stream)
 
 
-def decode(info: Info, d_blob, d_out, status=None, stream=None) -> None:
+def decode(info: Info, d_blob, d_out, status=None, stream=None, blob_size: Optional[int] = None) -> None:
     """Asynchronously decode one blob already in device memory into d_out
-    (torch uint8 CUDA tensors or raw device pointers) on ``stream``."""
-    _check(_lib.ecf8_decode(ctypes.byref(info), _ptr(d_blob), _ptr(d_out), info.n, _ptr(status),
+    (torch uint8 CUDA tensors or raw device pointers) on ``stream``.  The
+    bytes readable at d_blob are the tensor's size, or ``blob_size`` (which a
+    raw pointer needs; it defaults to the blob's own size)."""
+    size = _nbytes(d_blob, info.blob_bytes) if blob_size is None else int(blob_size)
+    _check(_lib.ecf8_decode(ctypes.byref(info), _ptr(d_blob), size, _ptr(d_out), info.n, _ptr(status),
                             _stream(stream)), "ecf8_decode")
 
 
@@ -305,6 +324,7 @@ def make_batch(items: Sequence[BatchItem]):
         keep.append(it.info)
         arr[i].info = ctypes.pointer(it.info)
         arr[i].d_blob = _ptr(it.d_blob)
+        arr[i].blob_size = _nbytes(it.d_blob, it.info.blob_bytes)
         arr[i].d_out = _ptr(it.d_out)
     return arr, keep
 
@@ -370,6 +390,7 @@ class Pipeline:
                 self._keep.append(t.info)
                 tarr[i].info = ctypes.pointer(t.info)
                 tarr[i].d_blob = _ptr(t.d_blob)
+                tarr[i].blob_size = _nbytes(t.d_blob, t.info.blob_bytes)
                 tarr[i].out_offset = int(t.out_offset)
             self._keep.append(tarr)
             larr[l].tensors = tarr

@@ -27,7 +27,9 @@
 //  * exponents are parked 4 bits each in lane-private shared memory, then
 //    funnel-shifted into a 32-weight-aligned stage; 16 bytes of stage plus a
 //    16-byte nibble load become 32 output bytes (byte-permute + 3-input
-//    logic), and consecutive lanes store consecutive 32-byte vectors.
+//    logic: the blob's nibble words put each weight's sign and mantissa
+//    where its output byte wants them, or one rotate away), and consecutive
+//    lanes store consecutive 32-byte vectors.
 //  * CTAs are persistent, one per SM.  A launch puts the wide-table tensors on
 //    CTAs [0, split) and the rest on the others; within each part every CTA
 //    takes a contiguous run of groups of equal estimated cost.  Every warp
@@ -65,9 +67,22 @@ constexpr int kMaxCodes = kSpanBits * kT;      // codes one group can hold: 8192
 constexpr int kStageWords = kMaxCodes / 8 + 8; // + alignment slack
 constexpr int kStagePhys = kStageWords + 2 * (kStageWords / 32 + 1) + 2;  // 2 pad words per 32
 
-constexpr int kWarps = 16;                     // warps per CTA
+// Tuning knobs (compile-time; the defaults are the measured best on B200).
+#ifndef ECF8_WARPS
+#define ECF8_WARPS 16
+#endif
+#ifndef ECF8_NIB_PREFETCH
+#define ECF8_NIB_PREFETCH 4
+#endif
+#ifndef ECF8_PREFETCH_NEXT
+#define ECF8_PREFETCH_NEXT 1
+#endif
+
+constexpr int kWarps = ECF8_WARPS;             // warps per CTA
 constexpr int kThreads = 32 * kWarps;
-constexpr int kND = 4;                         // 32-weight nibble blocks a lane prefetches in registers
+constexpr int kND = ECF8_NIB_PREFETCH;         // 32-weight nibble blocks a lane prefetches in registers
+constexpr int kNDA = kND > 0 ? kND : 1;        // their array size
+constexpr bool kPrefetchNext = ECF8_PREFETCH_NEXT != 0;  // fetch the next group's inputs during this one
 constexpr int kStates = 16;                    // tree nodes (<= 15 for 16 values) + the error state
 constexpr int kError = kStates - 1;
 
@@ -266,17 +281,16 @@ __device__ __forceinline__ uint32_t nidx(uint32_t w, uint32_t e, uint32_t k) {
 
 // ---------------------------------------------------------------- assembly
 
-__device__ __forceinline__ uint32_t bsel(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
-
 // 8 weights: E = their exponents, 4 bits each in order; N = their nibble
-// word (weight k<4 in byte k low half, weight 4+k in byte k high half).
+// word (byte k: weight k's sign in bit 7 and mantissa in bits 0-2, weight
+// 4+k's mantissa in bits 4-6, weight 4+((k+3)%4)'s sign in bit 3), so
+// weights 0-3 take N and weights 4-7 take N rotated right by 4, each masked
+// to bits 7 and 0-2 of every byte.
 __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, uint32_t& hi) {
   const uint32_t ev = (E << 3) & 0x78787878u;  // e0 e2 e4 e6 at bits 3-6 of bytes 0-3
   const uint32_t od = (E >> 1) & 0x78787878u;  // e1 e3 e5 e7
-  const uint32_t n_lo = bsel(0x80808080u, N << 4, N);  // sign to bit 7, mantissa in bits 0-2
-  const uint32_t n_hi = bsel(0x80808080u, N, N >> 4);
-  lo = __byte_perm(ev, od, 0x5140) | (n_lo & 0x87878787u);
-  hi = __byte_perm(ev, od, 0x7362) | (n_hi & 0x87878787u);
+  lo = __byte_perm(ev, od, 0x5140) | (N & 0x87878787u);
+  hi = __byte_perm(ev, od, 0x7362) | (__funnelshift_r(N, N, 4) & 0x87878787u);
 }
 
 // 32 weights from their exponents (4 words, 8 per word) and nibbles (16
@@ -304,6 +318,17 @@ __device__ __forceinline__ uint4 stage32(const uint32_t* stage, uint32_t d) {
   const uint2* st = reinterpret_cast<const uint2*>(stage);
   const uint2 a = st[sunit<kW>(2 * d)], b = st[sunit<kW>(2 * d + 1)];
   return make_uint4(a.x, a.y, b.x, b.y);
+}
+
+// The walk's packer step: when the accumulator has filled a word (sh >= 32),
+// park it as the lane's next private word and keep the carry.
+__device__ __forceinline__ void park(uint32_t& sh, uint32_t* priv, uint32_t& words, uint32_t& acc, uint32_t carry,
+                                     int32_t* status) {
+  const bool full = sh >= 32;
+  if (full && in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
+  words += full ? 1u : 0u;
+  acc = full ? carry : acc;
+  sh -= full ? 32u : 0u;
 }
 
 // ---------------------------------------------------------------- one group per warp
@@ -353,7 +378,7 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   const uint32_t units = offsets_ok ? (uint32_t)(((off0 & 31) + (off1 - off0) + 15) >> 4) : 0;
   const uint32_t blocks = (units + 1) >> 1;  // 32-weight blocks: 16 nibble bytes each
   const uint4* nib = reinterpret_cast<const uint4*>(dt->nibbles) + (off0 >> 5);
-  uint4 nv[kND];
+  uint4 nv[kNDA];
 #pragma unroll
   for (int j = 0; j < kND; ++j)
     if (lane + 32 * j < blocks && in_bounds((off0 >> 5) + lane + 32 * j < (n + 31) / 32, status))
@@ -408,12 +433,7 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
       acc |= e.x << sh;
       const uint32_t carry = __funnelshift_l(e.x, 0u, sh);
       sh += e.y >> 8;
-      if (sh >= 32) {
-        if (in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
-        ++words;
-        acc = carry;
-        sh -= 32;
-      }
+      park(sh, priv, words, acc, carry, status);
     }
   } else {
     // two bytes per packing step: each ends at most 4 codes (16 bits), so a
@@ -431,12 +451,7 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
       acc |= p << sh;
       const uint32_t carry = __funnelshift_l(p, 0u, sh);
       sh += n1 + (e2 >> 24);
-      if (sh >= 32) {
-        if (in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
-        ++words;
-        acc = carry;
-        sh -= 32;
-      }
+      park(sh, priv, words, acc, carry, status);
     }
   }
   if (sh && in_bounds(words < (uint32_t)kPrivWords, status)) priv[32 * words] = acc;
@@ -447,8 +462,8 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
   const uint32_t cnt = bad ? 0 : emitted - extra;
 
   // the rest of a group of many short codes, once the walk's registers are free
-  uint4 nv2[kND];
-  if (kW == kWide && blocks > 32u * kND) {
+  uint4 nv2[kNDA];
+  if (kND > 0 && kW == kWide && blocks > 32u * kND) {
 #pragma unroll
     for (int j = 0; j < kND; ++j)
       if (lane + 32 * (kND + j) < blocks && in_bounds((off0 >> 5) + lane + 32 * (kND + j) < (n + 31) / 32, status))
@@ -525,7 +540,7 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     if (2 * d + 2 <= end_full && (j > 0 || 2 * d >= first_full))  // first_full <= 2
       if (in_bounds(base + 32ull * d + 32 <= n, status)) put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), nv[j]);
   }
-  if (kW == kWide && end_full > 64u * kND) {
+  if (kND > 0 && kW == kWide && end_full > 64u * kND) {
 #pragma unroll
     for (int j = 0; j < kND; ++j) {
       const uint32_t d = lane + 32 * (kND + j);
@@ -534,7 +549,8 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     }
   }
   for (uint32_t d = lane + 32 * (kW == kWide ? 2 * kND : kND); 2 * d + 2 <= end_full; d += 32)
-    if (in_bounds(base + 32ull * d + 32 <= n, status)) put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), __ldg(nib + d));
+    if ((kND > 0 || 2 * d >= first_full) && in_bounds(base + 32ull * d + 32 <= n, status))
+      put32(out + base + 32ull * d, a32, stage32<kW>(stage, d), __ldg(nib + d));
   {
     // a whole unit whose block partner is not whole: unit first_full when it
     // is odd (lane 0), unit end_full - 1 when end_full is odd (lane 1)
@@ -557,8 +573,9 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
       const uint32_t i = 16 * ru + (lane & 15);
       const uint32_t e = (stage[sidx<kW>(i >> 3)] >> (4 * (i & 7))) & 15u;
       const uint32_t k = lane & 7;
-      const uint32_t v = (rw >> (8 * (k & 3) + ((k & 4) ? 4 : 0))) & 15u;
-      if (in_bounds(p < n, status)) out[p] = (uint8_t)(((v >> 3) << 7) | (e << 3) | (v & 7u));
+      const uint32_t half = k < 4 ? rw : __funnelshift_r(rw, rw, 4);
+      const uint32_t v = (half >> (8 * (k & 3))) & 0x87u;
+      if (in_bounds(p < n, status)) out[p] = (uint8_t)(v | (e << 3));
     }
   }
   __syncwarp();  // the stage and private words are reused by this warp's next group
@@ -632,13 +649,14 @@ __device__ __forceinline__ void decode_run(const DevTensor* table, int count, ui
     uint32_t g = g0 + warp;
     if (g < g1) {
       GroupIn in;
-      fetch_group(dt, g - tb, in);
+      if (kPrefetchNext) fetch_group(dt, g - tb, in);
       for (; g < g1; g += kWarps) {
         GroupIn nx;
         const bool more = g + kWarps < g1;
-        if (more) fetch_group(dt, g + kWarps - tb, nx);
+        if (!kPrefetchNext) fetch_group(dt, g - tb, in);
+        else if (more) fetch_group(dt, g + kWarps - tb, nx);
         process_group<kW>(dt, g - tb, in, sm, wa, status);
-        if (more) in = nx;
+        if (kPrefetchNext && more) in = nx;
       }
     }
     g0 = g1;
@@ -727,10 +745,9 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 int check_info(const ecf8_info* info) {
   if (!info) return ECF8_ERR_ARG;
-  if (info->lut_bits != kLutBits) return ECF8_ERR_UNSUPPORTED;
   Layout L;
   if (!compute_layout(info->n, info->code_bits, info->chunk_bytes, info->group_chunks, &L)) return ECF8_ERR_FORMAT;
-  if (L.groups != info->n_groups || L.total != info->blob_bytes || L.lut_off != info->lut_off ||
+  if (L.groups != info->n_groups || L.total != info->blob_bytes ||
       L.gaps_off != info->gaps_off || L.groups_off != info->groups_off || L.stream_off != info->stream_off ||
       L.nib_off != info->nibbles_off)
     return ECF8_ERR_FORMAT;
@@ -796,7 +813,7 @@ int check_tensor(const ecf8_tensor& t, bool* skip) {
   if (t.info->chunk_bytes != (uint32_t)kC || t.info->group_chunks != (uint32_t)kT) return ECF8_ERR_UNSUPPORTED;
   *skip = t.info->n == 0;
   if (*skip) return ECF8_OK;
-  if (!t.d_blob || !t.d_out) return ECF8_ERR_ARG;
+  if (!t.d_blob || !t.d_out || t.blob_size < t.info->blob_bytes) return ECF8_ERR_ARG;
   if (!aligned16(t.d_blob) || !aligned16(t.d_out)) return ECF8_ERR_ALIGN;
   return ECF8_OK;
 }
@@ -918,11 +935,11 @@ int ecf8_layout_supported(uint32_t chunk_bytes, uint32_t group_chunks) {
   return chunk_bytes == (uint32_t)kC && group_chunks == (uint32_t)kT;
 }
 
-int ecf8_decode(const ecf8_info* info, const void* d_blob, uint8_t* d_out, size_t n, int32_t* d_status,
-                cudaStream_t s) {
+int ecf8_decode(const ecf8_info* info, const void* d_blob, size_t blob_size, uint8_t* d_out, size_t n,
+                int32_t* d_status, cudaStream_t s) {
   if (!info) return ECF8_ERR_ARG;
   if (n != info->n) return ECF8_ERR_ARG;
-  const ecf8_tensor one{info, d_blob, d_out};
+  const ecf8_tensor one{info, d_blob, blob_size, d_out};
   DevTensor t[1];
   Part part[2];
   int rc = build_table(&one, 1, t, part);
@@ -950,6 +967,11 @@ int ecf8_decode_batched_ctas(const ecf8_tensor* tensors, int count, void* d_work
   if (used == 0) return ECF8_OK;
   const DevTensor* d_table = nullptr;
   if (count > kInlineMax) {
+    // the descriptor copy below reads a temporary host array, which a captured
+    // graph would read again at replay, after the array is gone
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return ECF8_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return ECF8_ERR_CAPTURE;
     if (cudaMemcpyAsync(d_workspace, v.data(), sizeof(DevTensor) * used, cudaMemcpyHostToDevice, s) != cudaSuccess)
       return ECF8_ERR_CUDA;
     d_table = static_cast<const DevTensor*>(d_workspace);

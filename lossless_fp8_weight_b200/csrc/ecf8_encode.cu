@@ -3,15 +3,15 @@
 // The ECF8 walkthrough encodes per tensor in order: exponent histogram
 // (§3.1.1 step 1), Huffman code (step 2), canonical code table, bit-packed
 // code stream with per-chunk gaps and per-group offsets (§3.2.1), raw sign
-// and mantissa nibbles.  Here the histogram and every per-weight step run on
-// the GPU; only the 16-symbol code construction and the 16 KB header/table
-// prefix stay on the host.  Steps:
+// and mantissa nibbles.  Here the histogram and every
+// per-weight step run on the GPU; only the 16-symbol code construction and
+// the 128-byte header stay on the host.  Steps:
 //   histogram_kernel   exponent counts (16 per tensor)
 //   seg_bits_kernel    code bits of every 4096-weight segment
 //   scan_kernel        segment start bits (exclusive scan, one CTA)
 //   pack_kernel        the code stream, gaps and group offsets
 //   tail_kernel        offsets of groups that start past the stream end
-//   nibble_kernel      8 sign/mantissa nibbles per 32-bit word
+//   nibble_kernel      8 signs and mantissas per 32-bit word
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -35,7 +35,6 @@ struct Code {
 };
 
 __device__ __forceinline__ uint32_t exponent_of(uint32_t b) { return (b >> 3) & 15u; }
-__device__ __forceinline__ uint32_t nibble_of(uint32_t b) { return ((b >> 7) << 3) | (b & 7u); }
 
 // The 16 bytes of thread t's weights (zero past n).
 __device__ __forceinline__ void load16(const uint8_t* x, uint64_t n, uint64_t i0, uint8_t b[16]) {
@@ -210,20 +209,27 @@ __global__ void tail_kernel(PackArgs p, uint64_t groups) {
   }
 }
 
-// Nibbles: weight i in byte 4(i/8) + (i%4), low half if i%8 < 4.
+// Signs and mantissas of 8 weights per word: byte k = weight k's sign (bit
+// 7) and mantissa (bits 0-2), weight 4+k's mantissa (bits 4-6) and weight
+// 4+((k+3)%4)'s sign (bit 3).  Given the two little-endian words of the 8
+// bytes: a = weights 0-3, b = weights 4-7.
+__device__ __forceinline__ uint32_t nibble_word(uint32_t a, uint32_t b) {
+  const uint32_t rot = __funnelshift_l(b, b, 4);  // weight 4+k's sign to bit 3 of byte k+1 (mod 4)
+  return (a & 0x87878787u) | ((b << 4) & 0x70707070u) | (rot & 0x08080808u);
+}
+
 __global__ void nibble_kernel(const uint8_t* __restrict__ x, uint64_t n, uint32_t* nib, uint64_t words) {
   for (uint64_t w = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words; w += (uint64_t)gridDim.x * blockDim.x) {
     const uint64_t i = w * 8;
-    uint32_t v = 0;
+    uint2 q;
     if (i + 8 <= n) {
-      const uint2 q = *reinterpret_cast<const uint2*>(x + i);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        v |= (nibble_of((q.x >> (8 * k)) & 0xFFu) << (8 * k)) | (nibble_of((q.y >> (8 * k)) & 0xFFu) << (8 * k + 4));
+      q = *reinterpret_cast<const uint2*>(x + i);
     } else {
-      for (int k = 0; k < 8 && i + k < n; ++k) v |= nibble_of(x[i + k]) << (k < 4 ? 8 * k : 8 * (k - 4) + 4);
+      uint32_t v[2] = {0, 0};
+      for (int k = 0; k < 8 && i + k < n; ++k) v[k >> 2] |= (uint32_t)x[i + k] << (8 * (k & 3));
+      q = make_uint2(v[0], v[1]);
     }
-    nib[w] = v;
+    nib[w] = nibble_word(q.x, q.y);
   }
 }
 
@@ -276,13 +282,14 @@ int ecf8_encode_device(const uint8_t* d_fp8, size_t n, const uint64_t hist[16], 
   if (blob_cap < L.total) return ECF8_ERR_CAPACITY;
   const uint64_t segs = (n + kSeg - 1) / kSeg;
   if (n && (!d_workspace || workspace_bytes < ecf8_encode_device_workspace_size(n))) return ECF8_ERR_WORKSPACE;
+  if (n && !aligned16(d_workspace)) return ECF8_ERR_ALIGN;
   uint8_t* blob = static_cast<uint8_t*>(d_blob);
-  // header and decode table from the host (a pageable copy: the host buffer
-  // has been read when cudaMemcpyAsync returns), zeros up to the nibbles
-  std::vector<uint8_t> prefix((size_t)L.gaps_off);
+  // the header from the host (a pageable copy: the host buffer has been read
+  // when cudaMemcpyAsync returns), zeros up to the nibbles
+  std::vector<uint8_t> prefix((size_t)kHeaderBytes);
   write_blob_prefix(prefix.data(), L, cb, code);
   if (cudaMemcpyAsync(blob, prefix.data(), prefix.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemsetAsync(blob + L.gaps_off, 0, L.nib_off - L.gaps_off, s) != cudaSuccess)
+      cudaMemsetAsync(blob + kHeaderBytes, 0, L.nib_off - kHeaderBytes, s) != cudaSuccess)
     return ECF8_ERR_CUDA;
   if (n) {
     Code c;

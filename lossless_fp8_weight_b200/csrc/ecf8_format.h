@@ -1,4 +1,4 @@
-// Library-internal constants and layout arithmetic for the ECF8 blob (version 1),
+// Library-internal constants and layout arithmetic for the ECF8 blob (version 2),
 // shared by the host encoder (ecf8_host.cpp) and the decode kernels
 // (ecf8_decode.cu).  The layout itself is documented in include/ecf8.h.
 #pragma once
@@ -10,17 +10,13 @@
 namespace ecf8 {
 
 constexpr uint32_t kMagic = 0x38464345u;  // "ECF8"
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 constexpr uint32_t kHeaderBytes = 128;
-constexpr uint32_t kLutBits = 12;  // decode window
-constexpr uint32_t kLutEntries = 1u << kLutBits;
-constexpr uint32_t kLutMaxSyms = 6;  // codes per table entry
 constexpr uint32_t kSectionAlign = 256;
 
 struct Layout {
   uint64_t n, code_bits, groups;
   uint32_t C, T;
-  uint64_t lut_off, lut_bytes;
   uint64_t gaps_off, gaps_bytes;
   uint64_t groups_off, groups_bytes;
   uint64_t stream_off, stream_bytes;
@@ -41,13 +37,11 @@ inline bool compute_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t 
   L->groups = (code_bits + group_bits - 1) / group_bits;
   if (L->groups > 0xFFFFFFFFull) return false;
   const uint64_t chunks = L->groups * T;
-  L->lut_bytes = n ? 4ull * kLutEntries : 0;
   L->gaps_bytes = align_up((chunks + 7) / 8 * 4, 16);
   L->groups_bytes = 8 * (L->groups + 1);
   L->stream_bytes = n ? chunks * C + 16 : 0;
   L->nib_bytes = (n + 31) / 32 * 16;
-  L->lut_off = align_up(kHeaderBytes, kSectionAlign);
-  L->gaps_off = align_up(L->lut_off + L->lut_bytes, kSectionAlign);
+  L->gaps_off = align_up(kHeaderBytes, kSectionAlign);
   L->groups_off = align_up(L->gaps_off + L->gaps_bytes, kSectionAlign);
   L->stream_off = align_up(L->groups_off + L->groups_bytes, kSectionAlign);
   L->nib_off = align_up(L->stream_off + L->stream_bytes, kSectionAlign);
@@ -56,8 +50,8 @@ inline bool compute_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t 
 }
 
 // Host side of the device encoder (ecf8_host.cpp): checks the codebook
-// against the tensor's histogram and lays the blob out; writes the header and
-// decode-table section, bytes [0, gaps_off), the same as ecf8_encode does.
+// against the tensor's histogram and lays the blob out; writes the 128-byte
+// header, the same as ecf8_encode does.
 int prepare_blob(const ecf8_codebook* cb, const uint64_t hist[16], uint64_t n, uint32_t chunk_bytes,
                  uint32_t group_chunks, Layout* L, uint16_t code[16]);
 void write_blob_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t code[16]);

@@ -34,7 +34,21 @@ inline void store_le32(uint8_t* p, uint32_t v) { memcpy(p, &v, 4); }
 inline void store_le64(uint8_t* p, uint64_t v) { memcpy(p, &v, 8); }
 
 inline uint32_t exponent_of(uint8_t b) { return (b >> 3) & 15u; }
-inline uint32_t nibble_of(uint8_t b) { return ((uint32_t)(b >> 7) << 3) | (b & 7u); }
+
+// Signs and mantissas of 8 weights in one word, laid out for the decoder:
+// byte k holds weight k's sign (bit 7) and mantissa (bits 0-2), weight 4+k's
+// mantissa (bits 4-6), and weight 4+((k+3)%4)'s sign (bit 3).  A decoder then
+// takes weights 0-3 as word & 0x87878787 and weights 4-7 as the word rotated
+// right by 4 bits & 0x87878787, each byte ready to OR with its exponent << 3.
+inline uint32_t nibble_word(const uint8_t* b) {
+  uint32_t v = 0;
+  for (int k = 0; k < 4; ++k) {
+    v |= (uint32_t)(b[k] & 0x87u) << (8 * k);
+    v |= (uint32_t)(b[4 + k] & 7u) << (8 * k + 4);
+    v |= (uint32_t)(b[4 + k] >> 7) << (8 * ((k + 1) & 3) + 3);
+  }
+  return v;
+}
 
 // Per-range exponent histograms, one per thread range, so that the encoder can
 // also derive each range's bit length without a second pass.
@@ -161,35 +175,6 @@ bool canonical(const uint8_t* len, uint16_t* code) {
   return true;
 }
 
-// The 4096-entry multi-code decode table.  A first table holds, for every
-// 12-bit window, the code it starts with (if that code is <= 12 bits); the
-// entry then chains through it while the next code fits in the bits left.
-void build_table(const uint8_t* len, const uint16_t* code, uint32_t* table) {
-  static_assert(kLutBits == 12, "table built for 12-bit windows");
-  std::vector<uint8_t> first_sym(kLutEntries, 0xFF), first_len(kLutEntries, 0);
-  for (int s = 0; s < 16; ++s) {
-    const int l = len[s];
-    if (!l || l > (int)kLutBits) continue;
-    const uint32_t lo = (uint32_t)code[s] << (kLutBits - l), hi = lo + (1u << (kLutBits - l));
-    for (uint32_t w = lo; w < hi; ++w) {
-      first_sym[w] = (uint8_t)s;
-      first_len[w] = (uint8_t)l;
-    }
-  }
-  for (uint32_t p = 0; p < kLutEntries; ++p) {
-    uint32_t used = 0, cnt = 0, syms = 0;
-    while (cnt < kLutMaxSyms && used < kLutBits) {
-      const uint32_t w = (p << used) & (kLutEntries - 1);
-      const uint32_t l = first_len[w];
-      if (!l || l > kLutBits - used) break;
-      syms |= (uint32_t)first_sym[w] << (4 * cnt);
-      ++cnt;
-      used += l;
-    }
-    table[p] = used | (cnt << 4) | (syms << 8);
-  }
-}
-
 // Writes codes [i0, i1) starting at stream bit bit0, and the gap and group
 // offset of every chunk that starts in [bit0, bit1), where bit1 is the start of
 // code i1 (the stream end for the last range).  Words shared with the
@@ -239,10 +224,9 @@ void pack_range(const uint8_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t 
   for (; boundary < bit1 && chunk < chunks; boundary += chunk_bits, ++chunk) put_gap(chunk, bit1 - boundary, i1);
 }
 
-// The header and the decode-table section of a blob; bytes [0, gaps_off)
-// must already be zero.
-void write_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t* code, uint8_t max_len,
-                  uint32_t chunk_bytes, uint32_t group_chunks) {
+// The 128-byte header of a blob; those bytes must already be zero.
+void write_header(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, uint8_t max_len, uint32_t chunk_bytes,
+                  uint32_t group_chunks) {
   const uint64_t n = L.n;
   store_le32(blob + 0, kMagic);
   store_le32(blob + 4, kVersion);
@@ -251,21 +235,16 @@ void write_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const
   store_le32(blob + 24, chunk_bytes);
   store_le32(blob + 28, group_chunks);
   store_le32(blob + 32, (uint32_t)L.groups);
-  store_le32(blob + 36, kLutBits);
+  store_le32(blob + 36, 0);  // reserved
   store_le32(blob + 40, n ? max_len : 0);
   store_le32(blob + 44, kHeaderBytes);
-  store_le64(blob + 48, L.lut_off);
+  store_le64(blob + 48, 0);  // reserved
   store_le64(blob + 56, L.gaps_off);
   store_le64(blob + 64, L.groups_off);
   store_le64(blob + 72, L.stream_off);
   store_le64(blob + 80, L.nib_off);
   store_le64(blob + 88, L.total);
   memcpy(blob + 96, cb->len, 16);
-  if (n) {
-    std::vector<uint32_t> table(kLutEntries);
-    build_table(cb->len, code, table.data());
-    memcpy(blob + L.lut_off, table.data(), 4 * kLutEntries);
-  }
 }
 
 bool codebook_ok(const ecf8_codebook* cb, uint16_t* code_out) {
@@ -295,6 +274,7 @@ const char* ecf8_strerror(int code) {
     case ECF8_ERR_CUDA: return "CUDA runtime error";
     case ECF8_ERR_WORKSPACE: return "workspace missing or too small";
     case ECF8_ERR_TOO_MANY: return "more tensors than the no-allocation decode table holds";
+    case ECF8_ERR_CAPTURE: return "the call copies from host memory and its stream is capturing a graph";
     default: return "unknown error";
   }
 }
@@ -344,6 +324,14 @@ int ecf8_encoded_size(const uint64_t hist[16], size_t n, const ecf8_codebook* cb
   return ECF8_OK;
 }
 
+size_t ecf8_encoded_size_bound(size_t n, uint32_t chunk_bytes, uint32_t group_chunks) {
+  // every code is at most 16 bits long, so a stream never exceeds 16 n bits
+  if (n > (SIZE_MAX >> 5)) return 0;
+  Layout L;
+  if (!compute_layout(n, 16ull * n, chunk_bytes, group_chunks, &L)) return 0;
+  return (size_t)L.total;
+}
+
 int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t chunk_bytes, uint32_t group_chunks,
                 void* blob_v, size_t cap, size_t* blob_bytes) {
   if (!cb || !blob_v || !blob_bytes || (!fp8 && n)) return ECF8_ERR_ARG;
@@ -370,7 +358,7 @@ int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t 
 
   // zero everything but the nibble section, which is written whole below
   memset(blob, 0, L.nib_off);
-  write_prefix(blob, L, cb, code, max_len, chunk_bytes, group_chunks);
+  write_header(blob, L, cb, max_len, chunk_bytes, group_chunks);
 
   uint32_t* stream = reinterpret_cast<uint32_t*>(blob + L.stream_off);
   uint32_t* gaps = reinterpret_cast<uint32_t*>(blob + L.gaps_off);
@@ -389,21 +377,15 @@ int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t 
     if (c % group_chunks == 0) offs[c / group_chunks] = n;
   offs[L.groups] = n;
 
-  // nibbles: 8 weights per little-endian u32, weight k of 4 in byte k low half,
-  // weight 4 + k in byte k high half
+  // sign/mantissa: 8 weights per little-endian u32 (see nibble_word)
   uint32_t* nib = reinterpret_cast<uint32_t*>(blob + L.nib_off);
   const long long words = (long long)(L.nib_bytes / 4);
 #pragma omp parallel for num_threads(parts) schedule(static)
   for (long long w = 0; w < words; ++w) {
     const size_t i = (size_t)w * 8;
-    uint32_t v = 0;
-    if (i + 8 <= n) {
-      for (int k = 0; k < 4; ++k)
-        v |= (nibble_of(fp8[i + k]) << (8 * k)) | (nibble_of(fp8[i + 4 + k]) << (8 * k + 4));
-    } else {
-      for (int k = 0; k < 8 && i + k < n; ++k) v |= nibble_of(fp8[i + k]) << (k < 4 ? 8 * k : 8 * (k - 4) + 4);
-    }
-    nib[w] = v;
+    uint8_t b[8] = {};
+    for (int k = 0; k < 8 && i + k < n; ++k) b[k] = fp8[i + k];
+    nib[w] = nibble_word(b);
   }
   *blob_bytes = L.total;
   return ECF8_OK;
@@ -413,13 +395,13 @@ int ecf8_blob_info(const void* blob_v, size_t size, ecf8_info* out) {
   if (!blob_v || !out) return ECF8_ERR_ARG;
   const uint8_t* b = static_cast<const uint8_t*>(blob_v);
   if (size < kHeaderBytes) return ECF8_ERR_FORMAT;
-  if (load_le32(b) != kMagic || load_le32(b + 4) != kVersion || load_le32(b + 36) != kLutBits ||
+  if (load_le32(b) != kMagic || load_le32(b + 4) != kVersion || load_le32(b + 36) != 0 ||
       load_le32(b + 44) != kHeaderBytes)
     return ECF8_ERR_FORMAT;
   Layout L;
   const uint64_t n = load_le64(b + 8), code_bits = load_le64(b + 16);
   if (!compute_layout(n, code_bits, load_le32(b + 24), load_le32(b + 28), &L)) return ECF8_ERR_FORMAT;
-  if (L.groups != load_le32(b + 32) || L.lut_off != load_le64(b + 48) || L.gaps_off != load_le64(b + 56) ||
+  if (L.groups != load_le32(b + 32) || load_le64(b + 48) != 0 || L.gaps_off != load_le64(b + 56) ||
       L.groups_off != load_le64(b + 64) || L.stream_off != load_le64(b + 72) || L.nib_off != load_le64(b + 80) ||
       L.total != load_le64(b + 88) || L.total > size)
     return ECF8_ERR_FORMAT;
@@ -436,15 +418,9 @@ int ecf8_blob_info(const void* blob_v, size_t size, ecf8_info* out) {
   if (max_len != load_le32(b + 40)) return ECF8_ERR_FORMAT;
   if (n && (!present || code_bits < n || code_bits > 16 * n)) return ECF8_ERR_FORMAT;
   if (!n && code_bits) return ECF8_ERR_FORMAT;
-  if (n) {
-    std::vector<uint32_t> table(kLutEntries);
-    build_table(info.len, code, table.data());
-    if (memcmp(table.data(), b + L.lut_off, 4 * kLutEntries) != 0) return ECF8_ERR_FORMAT;
-  }
   info.n = n;
   info.code_bits = code_bits;
   info.blob_bytes = L.total;
-  info.lut_off = L.lut_off;
   info.gaps_off = L.gaps_off;
   info.groups_off = L.groups_off;
   info.stream_off = L.stream_off;
@@ -452,7 +428,6 @@ int ecf8_blob_info(const void* blob_v, size_t size, ecf8_info* out) {
   info.chunk_bytes = L.C;
   info.group_chunks = L.T;
   info.n_groups = (uint32_t)L.groups;
-  info.lut_bits = kLutBits;
   info.max_len = max_len;
   *out = info;
   return ECF8_OK;
@@ -477,11 +452,11 @@ int prepare_blob(const ecf8_codebook* cb, const uint64_t hist[16], uint64_t n, u
   return ECF8_OK;
 }
 
-void write_blob_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t code[16]) {
-  memset(blob, 0, L.gaps_off);
+void write_blob_prefix(uint8_t* blob, const Layout& L, const ecf8_codebook* cb, const uint16_t[16]) {
+  memset(blob, 0, kHeaderBytes);
   uint8_t max_len = 0;
   for (int s = 0; s < 16; ++s) max_len = std::max(max_len, cb->len[s]);
-  write_prefix(blob, L, cb, code, max_len, L.C, L.T);
+  write_header(blob, L, cb, max_len, L.C, L.T);
 }
 
 }  // namespace ecf8

@@ -28,6 +28,7 @@ struct SlotState {
 struct LayerDesc {
   std::vector<ecf8_info> infos;
   std::vector<const void*> blobs;
+  std::vector<size_t> blob_sizes;
   std::vector<size_t> offsets;
 };
 
@@ -63,7 +64,7 @@ int enqueue(ecf8_pipeline* p, int m) {
   p->scratch.resize(L.infos.size());
   uint8_t* base = static_cast<uint8_t*>(p->slots[(size_t)s]);
   for (size_t i = 0; i < L.infos.size(); ++i)
-    p->scratch[i] = ecf8_tensor{&L.infos[i], L.blobs[i], base + L.offsets[i]};
+    p->scratch[i] = ecf8_tensor{&L.infos[i], L.blobs[i], L.blob_sizes[i], base + L.offsets[i]};
   int rc = ecf8_decode_batched_ctas(p->scratch.data(), (int)p->scratch.size(), p->workspace, p->workspace_bytes,
                                     p->status, p->decode, p->max_ctas);
   if (rc) return rc;
@@ -90,6 +91,7 @@ int ecf8_pipeline_create(const ecf8_layer* layers, int n_layers, void* const* d_
     for (int i = 0; i < L.count; ++i) {
       const ecf8_layer_tensor& t = L.tensors[i];
       if (!t.info) return ECF8_ERR_ARG;
+      if (t.info->n && t.blob_size < t.info->blob_bytes) return ECF8_ERR_ARG;
       if ((t.out_offset & 15) != 0) return ECF8_ERR_ALIGN;
       if (t.out_offset > slot_bytes || t.info->n > slot_bytes - t.out_offset) return ECF8_ERR_ARG;
     }
@@ -108,6 +110,7 @@ int ecf8_pipeline_create(const ecf8_layer* layers, int n_layers, void* const* d_
       const ecf8_layer_tensor& t = layers[l].tensors[i];
       D.infos.push_back(*t.info);
       D.blobs.push_back(t.d_blob);
+      D.blob_sizes.push_back(t.blob_size);
       D.offsets.push_back(t.out_offset);
     }
   }

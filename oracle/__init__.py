@@ -6,8 +6,7 @@ import this package; the library under ``lossless_fp8_weight_b200/`` never does.
 
 The oracle fixes what the GPU path must compute: ``decode(encode(x)) == x`` byte
 for byte (ECF8 walkthrough p1 §1; arXiv 2510.02676 abstract), with the blob
-layout, code construction and decode table spelled out step by step in the C
-source.
+layout and the code construction spelled out step by step in the C source.
 """
 from __future__ import annotations
 
@@ -22,8 +21,6 @@ _SRC = os.path.join(_HERE, "ecf8_oracle.c")
 _SO = os.path.join(_HERE, "libecf8_oracle.so")
 
 NSYM = 16
-LUT_BITS = 12
-LUT_MAX_SYMS = 6
 
 
 _BF16_SRC = os.path.join(_HERE, "bf16_oracle.c")
@@ -51,8 +48,6 @@ def _load():
         lib.oracle_package_merge_lengths.argtypes = [p, i32, p]
         lib.oracle_code_lengths.argtypes = [p, i32, p]
         lib.oracle_canonical_codes.argtypes = [p, p]
-        lib.oracle_lut_entry.argtypes = [p, u32]
-        lib.oracle_lut_entry.restype = u32
         lib.oracle_encoded_size.argtypes = [p, u64, p, u32, u32]
         lib.oracle_encoded_size.restype = u64
         lib.oracle_encode.argtypes = [p, u64, p, u32, u32, p, u64, ctypes.POINTER(u64)]
@@ -128,11 +123,6 @@ def canonical_codes(lengths) -> np.ndarray:
     return out
 
 
-def lut_entry(lengths, pattern: int) -> int:
-    ln = _u8(lengths)
-    return int(_load().oracle_lut_entry(ln.ctypes.data, pattern))
-
-
 def encode(x, lengths=None, chunk_bytes: int = 32, group_chunks: int = 32, max_len: int = 16) -> np.ndarray:
     """Blob for ``x`` (uint8 E4M3 bytes).  Lengths default to the code built
     from ``x``'s own exponent histogram."""
@@ -168,8 +158,8 @@ def decode_into(blob, out: np.ndarray) -> int:
 
 
 def check_index(blob) -> int:
-    """0 when the blob's gaps, group offsets and decode table equal the ones the
-    serial walk recomputes; 1 table, 2 gap, 3 offset, 4 stream, -1 header."""
+    """0 when the blob's gaps and group offsets equal the ones the serial walk
+    recomputes; 2 gap, 3 offset, 4 stream, -1 header."""
     b = _u8(blob)
     return int(_load().oracle_check_index(b.ctypes.data, b.size))
 
@@ -181,8 +171,8 @@ def blob_header(blob) -> dict:
     u64 = lambda o: int(b[o:o + 8].view("<u8")[0])  # noqa: E731
     return {
         "magic": u32(0), "version": u32(4), "n": u64(8), "code_bits": u64(16),
-        "chunk_bytes": u32(24), "group_chunks": u32(28), "n_groups": u32(32), "lut_bits": u32(36),
-        "max_len": u32(40), "header_bytes": u32(44), "lut_off": u64(48), "gaps_off": u64(56),
+        "chunk_bytes": u32(24), "group_chunks": u32(28), "n_groups": u32(32), "reserved": u32(36),
+        "max_len": u32(40), "header_bytes": u32(44), "reserved48": u64(48), "gaps_off": u64(56),
         "groups_off": u64(64), "stream_off": u64(72), "nibbles_off": u64(80), "total": u64(88),
         "lengths": b[96:112].copy(),
     }

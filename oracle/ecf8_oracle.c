@@ -27,11 +27,13 @@
  *    the stream (bit code_bits) counts as a start, so a chunk that begins
  *    inside the last code points past it; chunks beyond the end hold 0.
  *  - group g = T chunks; off[g] = number of codes starting before bit 8CTg.
- *  - nibbles: weight i lives in byte 4(i/8) + (i mod 4), low half if
- *    i mod 8 < 4, high half otherwise.
- *  - decode table (p1 §3.1.2, redesigned): 2^12 32-bit entries; entry for a
- *    12-bit window = greedy decode of at most 6 codes that lie wholly in it:
- *    bits 0-3 total length, 4-6 count, 8+4j symbol j.  0 if none fits.
+ *  - sign/mantissa nibbles, 8 weights per little-endian 32-bit word w: for
+ *    k = 0..3, byte k holds weight 8w+k's sign in bit 7 and mantissa in bits
+ *    0-2, weight 8w+4+k's mantissa in bits 4-6, and in bit 3 the sign of
+ *    weight 8w+4+((k+3) mod 4), i.e. weight 8w+4+k's sign sits in bit 3 of
+ *    byte (k+1) mod 4.  Four bits per weight, as the pages' nibble array.
+ *  - no decode table in the blob: the code lengths in the header are the
+ *    codebook, and a decoder derives whatever table it uses from them.
  *
  * Parity pins live in tests/test_oracle_pins.py.  Functions whose result has
  * no pin are marked "parity unpinned" (none at present).
@@ -41,11 +43,9 @@
 #include <string.h>
 
 #define NSYM 16
-#define LUT_BITS 12
-#define LUT_MAX_SYMS 6
 #define HEADER_BYTES 128
 #define MAGIC 0x38464345u /* bytes 'E' 'C' 'F' '8' */
-#define VERSION 1u
+#define VERSION 2u
 
 /* ---------- little-endian field access ---------- */
 static uint32_t rd32(const uint8_t* p) {
@@ -216,34 +216,11 @@ static int match_code(const uint8_t* len, const uint32_t* code, int (*bit)(const
 }
 
 static int stream_bit(const void* src, uint64_t i) { return get_bit((const uint8_t*)src, i); }
-static int window_bit(const void* src, uint64_t i) { /* bit i of a 12-bit window, MSB first */
-  uint32_t p = *(const uint32_t*)src;
-  return (int)((p >> (LUT_BITS - 1 - i)) & 1u);
-}
-
-/* ---------- decode table entry (p1 §3.1.2, one-level multi-symbol reading) ---------- */
-uint32_t oracle_lut_entry(const uint8_t* len, uint32_t pattern) {
-  uint32_t code[NSYM];
-  oracle_canonical_codes(len, code);
-  uint32_t entry = 0;
-  uint64_t pos = 0;
-  int count = 0;
-  while (count < LUT_MAX_SYMS) {
-    int used = 0;
-    int s = match_code(len, code, window_bit, &pattern, pos, LUT_BITS - pos, &used);
-    if (s < 0) break;
-    entry |= (uint32_t)s << (8 + 4 * count);
-    count += 1;
-    pos += (uint64_t)used;
-  }
-  return entry | ((uint32_t)count << 4) | (uint32_t)pos;
-}
-
 /* ---------- blob layout ---------- */
 typedef struct {
   uint64_t n, code_bits, groups;
   uint32_t C, T;
-  uint64_t lut_off, lut_size, gaps_off, gaps_size, groups_off, groups_size;
+  uint64_t gaps_off, gaps_size, groups_off, groups_size;
   uint64_t stream_off, stream_size, nib_off, nib_size, total;
 } layout_t;
 
@@ -255,15 +232,13 @@ static int make_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t T, l
   L->n = n; L->code_bits = code_bits; L->C = C; L->T = T;
   uint64_t group_bits = 8ull * C * T;
   L->groups = (code_bits + group_bits - 1) / group_bits;
-  L->lut_size = n ? 4ull << LUT_BITS : 0;
   uint64_t chunks = L->groups * T;
   L->gaps_size = (chunks + 7) / 8 * 4;
   L->gaps_size = (L->gaps_size + 15) / 16 * 16;
   L->groups_size = 8 * (L->groups + 1);
   L->stream_size = n ? L->groups * T * C + 16 : 0;
   L->nib_size = (n + 31) / 32 * 16;
-  L->lut_off = up256(HEADER_BYTES);
-  L->gaps_off = up256(L->lut_off + L->lut_size);
+  L->gaps_off = up256(HEADER_BYTES);
   L->groups_off = up256(L->gaps_off + L->gaps_size);
   L->stream_off = up256(L->groups_off + L->groups_size);
   L->nib_off = up256(L->stream_off + L->stream_size);
@@ -305,20 +280,16 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
   wr32(blob + 24, C);
   wr32(blob + 28, T);
   wr32(blob + 32, (uint32_t)L.groups);
-  wr32(blob + 36, LUT_BITS);
+  wr32(blob + 36, 0); /* reserved */
   wr32(blob + 40, (uint32_t)max_len);
   wr32(blob + 44, HEADER_BYTES);
-  wr64(blob + 48, L.lut_off);
+  wr64(blob + 48, 0); /* reserved */
   wr64(blob + 56, L.gaps_off);
   wr64(blob + 64, L.groups_off);
   wr64(blob + 72, L.stream_off);
   wr64(blob + 80, L.nib_off);
   wr64(blob + 88, L.total);
   for (int s = 0; s < NSYM; ++s) blob[96 + s] = len[s];
-
-  /* decode table */
-  if (n)
-    for (uint32_t p = 0; p < (1u << LUT_BITS); ++p) wr32(blob + L.lut_off + 4 * p, oracle_lut_entry(len, p));
 
   /* code stream, one bit at a time, and the code start positions it implies */
   uint8_t* stream = blob + L.stream_off;
@@ -351,12 +322,20 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
     if (next_chunk % T == 0) wr64(offs + 8 * (next_chunk / T), n);
   wr64(offs + 8 * L.groups, n);
 
-  /* sign + mantissa nibbles */
+  /* sign + mantissa nibbles, bit by bit at the places the layout gives them */
   uint8_t* nib = blob + L.nib_off;
   for (uint64_t i = 0; i < n; ++i) {
-    uint64_t byte = 4 * (i / 8) + (i % 4);
     int v = oracle_nibble(x[i]);
-    nib[byte] |= (uint8_t)((i % 8) < 4 ? v : v << 4);
+    int sign = (v >> 3) & 1, mant = v & 7;
+    uint64_t word = 4 * (i / 8);
+    int r = (int)(i % 8);
+    if (r < 4) {
+      nib[word + r] |= (uint8_t)((sign << 7) | mant);
+    } else {
+      int k = r - 4;
+      nib[word + k] |= (uint8_t)(mant << 4);
+      nib[word + (k + 1) % 4] |= (uint8_t)(sign << 3);
+    }
   }
   *size = L.total;
   return 0;
@@ -365,10 +344,10 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
 /* ---------- header parse ---------- */
 static int read_layout(const uint8_t* blob, uint64_t size, layout_t* L, uint8_t* len) {
   if (size < HEADER_BYTES || rd32(blob) != MAGIC || rd32(blob + 4) != VERSION) return -1;
-  if (rd32(blob + 36) != LUT_BITS || rd32(blob + 44) != HEADER_BYTES) return -1;
+  if (rd32(blob + 36) != 0 || rd32(blob + 44) != HEADER_BYTES) return -1;
   uint64_t n = rd64(blob + 8), code_bits = rd64(blob + 16);
   if (make_layout(n, code_bits, rd32(blob + 24), rd32(blob + 28), L) != 0) return -1;
-  if (L->groups != rd32(blob + 32) || L->lut_off != rd64(blob + 48) || L->gaps_off != rd64(blob + 56) ||
+  if (L->groups != rd32(blob + 32) || rd64(blob + 48) != 0 || L->gaps_off != rd64(blob + 56) ||
       L->groups_off != rd64(blob + 64) || L->stream_off != rd64(blob + 72) ||
       L->nib_off != rd64(blob + 80) || L->total != rd64(blob + 88) || L->total > size)
     return -1;
@@ -376,7 +355,7 @@ static int read_layout(const uint8_t* blob, uint64_t size, layout_t* L, uint8_t*
   return 0;
 }
 
-/* ---------- step 10: bit-serial decode; ignores gaps, offsets and the table ---------- */
+/* ---------- step 10: bit-serial decode; ignores gaps and offsets ---------- */
 int oracle_decode(const uint8_t* blob, uint64_t size, uint8_t* out, uint64_t n) {
   layout_t L;
   uint8_t len[NSYM];
@@ -392,23 +371,27 @@ int oracle_decode(const uint8_t* blob, uint64_t size, uint8_t* out, uint64_t n) 
     int e = match_code(len, code, stream_bit, stream, pos, L.code_bits - pos, &used);
     if (e < 0) return -5;
     pos += (uint64_t)used;
-    uint8_t byte = nib[4 * (i / 8) + (i % 4)];
-    int v = (i % 8) < 4 ? (byte & 15) : (byte >> 4);
-    out[i] = oracle_join(e, v);
+    const uint8_t* word = nib + 4 * (i / 8);
+    int r = (int)(i % 8), sign, mant;
+    if (r < 4) {
+      sign = (word[r] >> 7) & 1;
+      mant = word[r] & 7;
+    } else {
+      mant = (word[r - 4] >> 4) & 7;
+      sign = (word[(r - 3) % 4] >> 3) & 1;
+    }
+    out[i] = oracle_join(e, (sign << 3) | mant);
   }
   return pos == L.code_bits ? 0 : -6;
 }
 
-/* ---------- recompute gaps, group offsets and the table by the serial walk ---------- */
+/* ---------- recompute gaps and group offsets by the serial walk ---------- */
 int oracle_check_index(const uint8_t* blob, uint64_t size) {
   layout_t L;
   uint8_t len[NSYM];
   uint32_t code[NSYM];
   if (read_layout(blob, size, &L, len) != 0) return -1;
   if (oracle_canonical_codes(len, code) != 0) return -1;
-  if (L.n)
-    for (uint32_t p = 0; p < (1u << LUT_BITS); ++p)
-      if (rd32(blob + L.lut_off + 4 * p) != oracle_lut_entry(len, p)) return 1;
   const uint8_t* stream = blob + L.stream_off;
   uint64_t chunk_bits = 8ull * L.C, chunks = L.groups * L.T, c = 0, pos = 0;
   for (uint64_t i = 0; i <= L.n + 1; ++i) {

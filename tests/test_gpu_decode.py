@@ -90,8 +90,9 @@ def test_two_symbols(env):
 
 
 def test_deepest_code_takes_the_long_path(env):
-    """Fibonacci exponent counts: codes of 13-15 bits, longer than the 12-bit
-    table window, decode through the canonical fallback."""
+    """Fibonacci exponent counts: codes of up to 15 bits, which span two or
+    three stream bytes; the byte state machine carries them across byte steps
+    through its tree nodes like any shorter code."""
     fib = [1, 1]
     while len(fib) < 16:
         fib.append(fib[-1] + fib[-2])
@@ -147,6 +148,9 @@ def test_argument_errors(env):
     with pytest.raises(L.Ecf8Error) as e:
         L.decode(L.blob_info(odd), _to_dev(torch, odd), out)
     assert e.value.code == -6
+    with pytest.raises(L.Ecf8Error) as e:  # a device buffer shorter than the blob
+        L.decode(info, d[16:16 + info.blob_bytes - 1], out)
+    assert e.value.code == -1
 
 
 # ------------------------------------------------------------------ corrupt blobs
@@ -164,7 +168,8 @@ def test_corrupt_gap_is_reported_and_contained(env):
     blob = oracle.encode(x)
     hd = oracle.blob_header(blob)
     _, status, intact = _corrupt_and_decode(env, blob, hd["gaps_off"] + 40, 0x30)
-    assert intact and status & 1
+    assert intact and status & 3  # the group's code count no longer matches its offsets, or no code
+
 
 
 def test_corrupt_offsets_are_reported_and_contained(env):
@@ -244,6 +249,49 @@ def test_batched_without_workspace_fails_loudly(env):
     with pytest.raises(L.Ecf8Error) as e:
         _batched(env, blobs, workspace=False)
     assert e.value.code == -8
+
+
+def test_batched_decode_in_a_captured_graph(env):
+    """A batch that travels in the launch's parameters (up to 64 tensors)
+    copies nothing from the host, so it records into a CUDA graph and replays
+    to the same bytes; a larger batch copies its descriptors from a host
+    array and refuses capture (ECF8_ERR_CAPTURE) without enqueueing."""
+    L, torch = env
+    xs = [synth.single_normal_1k().tensors[0].generate(begin=7 * k, count=20_000 + 1000 * k) for k in range(5)]
+    blobs = [L.encode(x) for x in xs]
+    infos = [L.blob_info(b) for b in blobs]
+    d_blobs = [_to_dev(torch, b) for b in blobs]
+    outs = [torch.zeros(i.n, dtype=torch.uint8, device="cuda") for i in infos]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    batch = L.make_batch([L.BatchItem(i, b, o) for i, b, o in zip(infos, d_blobs, outs)])
+    side = torch.cuda.Stream()
+    L.decode_batched(batch, status=status, stream=side)  # first call outside capture: kernel attributes
+    torch.cuda.synchronize()
+    for o in outs:
+        o.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        L.decode_batched(batch, status=status, stream=side)
+    g.replay()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for x, o in zip(xs, outs):
+        assert np.array_equal(o.cpu().numpy(), x)
+
+    big = [L.encode(np.full(100, 0x38, np.uint8)) for _ in range(L.BATCH_INLINE_MAX + 1)]
+    big_infos = [L.blob_info(b) for b in big]
+    big_dev = [_to_dev(torch, b) for b in big]
+    big_out = [torch.empty(100, dtype=torch.uint8, device="cuda") for _ in big]
+    ws = torch.empty(L.batched_workspace_size(len(big)), dtype=torch.uint8, device="cuda")
+    big_batch = L.make_batch([L.BatchItem(i, b, o) for i, b, o in zip(big_infos, big_dev, big_out)])
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=side):
+        with pytest.raises(L.Ecf8Error) as e:
+            L.decode_batched(big_batch, workspace=ws, status=status, stream=side)
+    assert e.value.code == -10
+    L.decode_batched(big_batch, workspace=ws, status=status)  # outside capture it runs
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0 and all((o.cpu().numpy() == 0x38).all() for o in big_out)
 
 
 def test_back_to_back_decodes_into_one_buffer_keep_stream_order(env):

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_function(L):
 
 def test_abi_version_and_strerror(L):
     so = ctypes.CDLL(L.library_path())
-    assert so.ecf8_abi_version() == 1
+    assert so.ecf8_abi_version() == 2
     so.ecf8_strerror.restype = ctypes.c_char_p
     assert so.ecf8_strerror(0) == b"ok"
     assert so.ecf8_strerror(-5).startswith(b"device pointer")
@@ -108,7 +108,7 @@ def test_blob_info_rejects_damage(L):
         with pytest.raises(L.Ecf8Error):
             L.blob_info(bad)
     bad = blob.copy()
-    bad[256 + 4 * 100] ^= 1  # decode table
+    bad[36] = 12  # the version-1 table field: version 2 reserves it as 0
     with pytest.raises(L.Ecf8Error):
         L.blob_info(bad)
     bad = blob.copy()
@@ -135,6 +135,31 @@ def test_layout_support_and_workspace_sizes(L):
     assert not L.layout_supported(4, 1)
     assert L.batched_workspace_size(1) == 0 and L.batched_workspace_size(64) == 0
     assert L.batched_workspace_size(65) == 65 * 96
+
+
+def test_encoded_size_bound_covers_every_input(L):
+    """The histogram-free bound holds for the worst inputs of every layout: the
+    16-bit-code tensor of a skewed 16-value code, uniform random bytes, and
+    sizes around the chunk and group boundaries."""
+    fib = [1, 1]
+    while len(fib) < 16:
+        fib.append(fib[-1] + fib[-2])
+    deep = np.repeat(np.arange(16, dtype=np.uint8) << 3, fib)
+    r = np.random.default_rng(17)
+    for C, T in [(32, 32), (4, 1), (16, 3), (64, 64)]:
+        for x in [deep, r.integers(0, 256, size=100_001).astype(np.uint8), np.zeros(1, np.uint8)]:
+            assert L.encode(x, chunk_bytes=C, group_chunks=T).size <= L.encoded_size_bound(x.size, C, T)
+        # all 16-bit codes: the largest stream any code allows
+        x = np.zeros(4097, np.uint8)
+        h = np.zeros(16, np.uint64)
+        h[0] = x.size
+        cb = L.Codebook()
+        cb.len[0] = 16
+        cb.code[0] = 0
+        size = ctypes.c_size_t(0)
+        assert L._lib.ecf8_encoded_size(h.ctypes.data, x.size, ctypes.byref(cb), C, T, ctypes.byref(size)) == 0
+        assert size.value == L.encoded_size_bound(x.size, C, T)
+    assert L.encoded_size_bound(10, 3, 1) == 0  # chunk bytes not a multiple of 4
 
 
 def test_compression_of_pages_like_weights(L):

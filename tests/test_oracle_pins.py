@@ -2,9 +2,9 @@
 the oracle's own code.
 
 Sources: ECF8 walkthrough ("ECF8 浮点数压缩技术") p1 §1 (bit-exact), §3.1.1
-(per-layer exponent statistics, optimal prefix code, length <= 16), §3.1.2
-(decode table), §3.2.1 (per-thread gap), §5.3 (gap synchronisation as the
-failure mode); arXiv 2510.02676 abstract (lossless, "no deviation").
+(per-layer exponent statistics, optimal prefix code, length <= 16), §3.2.1
+(per-thread gap and output position), §5.3 (gap synchronisation as the failure
+mode); arXiv 2510.02676 abstract (lossless, "no deviation").
 """
 import itertools
 import math
@@ -210,22 +210,20 @@ def test_two_symbols_stream_is_a_bitmap():
     bits += "0" * (-len(bits) % 32)
     want = np.array([int(bits[i:i + 32], 2) for i in range(0, len(bits), 32)], dtype=np.uint32)
     assert np.array_equal(words, want)
+    assert oracle.check_index(blob) == 0
 
 
 # ---------------------------------------------------------------- worked example (hand-derived)
 
 def _read_golden(name):
-    d = {"lut": []}
+    d = {}
     with open(os.path.join(GOLDEN, name)) as f:
         for line in f:
             line = line.strip()
             if not line or line.startswith("#"):
                 continue
             key, *vals = line.split()
-            if key == "lut":
-                d["lut"].append((int(vals[0], 16), int(vals[1], 16)))
-            else:
-                d[key] = vals
+            d[key] = vals
     return d
 
 
@@ -250,32 +248,39 @@ def test_hand_worked_example():
     assert [int(w) for w in go] == [int(v) for v in g["group_offsets"]]
     nb = blob[hd["nibbles_off"]:hd["nibbles_off"] + 16]
     assert [int(v) for v in nb] == [int(v, 16) for v in g["nibble_bytes"]]
-    lut = blob[hd["lut_off"]:hd["lut_off"] + 4 * 4096].view("<u4")
-    for pat, want in g["lut"]:
-        assert int(lut[pat]) == want, hex(pat)
+    assert hd["version"] == 2 and hd["reserved"] == 0 and hd["reserved48"] == 0
     assert np.array_equal(oracle.decode(blob, x.size), x)
 
 
-# ---------------------------------------------------------------- decode table
+# ---------------------------------------------------------------- nibble section
 
-def test_decode_table_entries_are_greedy_and_maximal():
-    """Each entry's codes spell exactly its first `used` bits, and either it holds
-    6 codes or no code fits in the bits left over -- this fixes every entry."""
-    for h in list(_random_hists(6, seed=21)) + [np.array([1, 1] + [0] * 14, dtype=np.uint64)]:
-        ln = oracle.code_lengths(h)
-        codes = oracle.canonical_codes(ln)
-        words = {s: format(int(codes[s]), f"0{int(ln[s])}b") for s in range(16) if ln[s]}
-        for pat in range(4096):
-            e = oracle.lut_entry(ln, pat)
-            used, cnt = e & 15, (e >> 4) & 7
-            syms = [(e >> (8 + 4 * j)) & 15 for j in range(cnt)]
-            assert e >> (8 + 4 * cnt) == 0 and (e >> 7) & 1 == 0
-            bits = format(pat, "012b")
-            spelled = "".join(words[s] for s in syms)
-            assert spelled == bits[:used] and len(spelled) == used
-            rest = bits[used:]
-            if cnt < 6:
-                assert not any(rest.startswith(w) for w in words.values())
+def test_nibble_layout_is_a_permutation_of_four_bits_per_weight():
+    """The pages keep sign and mantissa raw, 4 bits a weight: whatever the bit
+    order, each of a weight's 4 bits must land on its own bit of the nibble
+    section and no two weights may share one.  Found here by encoding single
+    set bits (one weight's sign or one mantissa bit) and locating the one bit
+    that lights up."""
+    n = 24  # three nibble words
+    base = np.full(n, 0x38, dtype=np.uint8)  # exponent 7 everywhere: the same code stream
+    seen = {}
+    ref = oracle.encode(base)
+    hd = oracle.blob_header(ref)
+    lo, hi = hd["nibbles_off"], hd["nibbles_off"] + 4 * (n // 8)
+    assert not ref[lo:hi].any()
+    for i in range(n):
+        for bit in (0x80, 0x01, 0x02, 0x04):  # sign, mantissa bits 0-2
+            x = base.copy()
+            x[i] |= bit
+            blob = oracle.encode(x)
+            assert np.array_equal(blob[:lo], ref[:lo])  # nothing but the nibbles changes
+            diff = np.unpackbits(blob[lo:hi] ^ ref[lo:hi], bitorder="little")
+            pos = np.flatnonzero(diff)
+            assert pos.size == 1, (i, bit)
+            p = int(pos[0])
+            assert p // 32 == i // 8  # weight i lives in word i // 8
+            assert p not in seen, (i, bit, seen.get(p))
+            seen[p] = (i, bit)
+    assert sorted(seen) == list(range(4 * n))
 
 
 # ---------------------------------------------------------------- round trip (the definition)
@@ -344,9 +349,6 @@ def test_corrupt_gap_and_offset_are_detected():
     bad = blob.copy()
     bad[hd["groups_off"] + 8] ^= 1
     assert oracle.check_index(bad) == 3
-    bad = blob.copy()
-    bad[hd["lut_off"] + 4 * 77] ^= 0x20
-    assert oracle.check_index(bad) == 1
     bad = blob.copy()
     bad[0] ^= 1
     with pytest.raises(ValueError):

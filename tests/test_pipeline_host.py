@@ -36,6 +36,7 @@ def _create(L, layers, slots, slot_bytes, depth, workspace=0, ws_bytes=0):
             keep.append(info)
             tarr[i].info = ctypes.pointer(info)
             tarr[i].d_blob = FAKE
+            tarr[i].blob_size = info.blob_bytes
             tarr[i].out_offset = off
         keep.append(tarr)
         larr[l].tensors = tarr
@@ -95,3 +96,20 @@ def test_null_and_empty_arguments(L):
     assert L._lib.ecf8_pipeline_acquire(None, 0, 0, ctypes.byref(ctypes.c_void_p())) == -1
     assert L._lib.ecf8_pipeline_release(None, 0, 0) == -1
     L._lib.ecf8_pipeline_destroy(None)  # a no-op
+
+
+def test_blob_buffers_must_hold_their_blobs(L):
+    (a,) = _infos(L, [1000])
+    n = 1
+    larr = (L.Layer * n)()
+    tarr = (L.LayerTensor * 1)()
+    tarr[0].info = ctypes.pointer(a)
+    tarr[0].d_blob = FAKE
+    tarr[0].blob_size = a.blob_bytes - 1
+    tarr[0].out_offset = 0
+    larr[0].tensors = tarr
+    larr[0].count = 1
+    sarr = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    h = ctypes.c_void_p()
+    assert L._lib.ecf8_pipeline_create(larr, n, sarr, 2, 4096, 1, 0, 0, 0, 0, 0, ctypes.byref(h)) == -1
+    assert not h.value

@@ -77,3 +77,14 @@ def test_noalloc_rejects_more_tensors_than_its_table(env):
         L.decode_batched_noalloc(items)
     assert e.value.code == -9
     assert L.launch_count() == before
+
+
+def test_noalloc_fills_its_table_to_the_last_entry(env):
+    """Exactly ECF8_NOALLOC_MAX_TENSORS tensors: every slot of the library's
+    table is written and read, the last one included."""
+    L, torch = env
+    r = np.random.default_rng(5)
+    spec = synth.single_normal_1k().tensors[0]
+    xs = [spec.generate(begin=int(r.integers(0, 1 << 20)), count=int(r.integers(1, 600)))
+          for _ in range(L.NOALLOC_MAX_TENSORS)]
+    _decode_both(L, torch, xs, [L.encode(x) for x in xs])
