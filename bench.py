@@ -1,17 +1,23 @@
 #!/usr/bin/env python3
 """ECF8 decode benchmark.
 
-One step = one batched decode launch over every tensor of the workload (the
-whole hot path: table load, chunk walk, scan, compaction, assembly, store),
-inputs resident in HBM.  Default workload: the seven projections of one
-Llama-3-8B decoder layer in FP8 E4M3 (q/o 4096x4096, k/v 1024x4096, gate/up
-14336x4096, down 4096x14336), weights symmetric alpha-stable alpha=1.8 scaled
-to max|w| = 448, one codebook per tensor: 218,103,808 bytes of FP8 out.
+Default workload: the Llama-3-70B weight set in FP8 E4M3 -- 80 decoder
+layers of seven projections (q/o 8192x8192, k/v 1024x8192, gate/up
+28672x8192, down 8192x28672), weights symmetric alpha-stable alpha=1.8 scaled
+to max|w| = 448, one codebook per tensor, 68,451,041,280 bytes of FP8 in all,
+held compressed in HBM and decoded layer by layer into ONE reused output
+buffer on one stream.  One step = the 80-layer loop: 80 batched decode
+launches (each the whole hot path: table build, chunk walk, scan,
+compaction, assembly, store), inputs resident in HBM.  The same JSON line
+carries the Llama-3-8B layer (one batched launch per step) and the
+256-expert MoE set (768 tensors, one batched launch) as extra fields.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-Multi-GPU (torchrun): every rank decodes its own copy of the layer (weak
-scaling; the decode has no exchange step), time = max over ranks.
+Other workloads (--workload llama3_8b_layer, sweep_<a>_<max>, moe, ...) time
+one batched launch per step.  Multi-GPU (torchrun): every rank decodes its
+own copy of the weights (weak scaling; the decode has no exchange step),
+time = max over ranks.
 """
 from __future__ import annotations
 
@@ -41,7 +47,12 @@ KERNEL_SRC = os.path.join(ROOT, "lossless_fp8_weight_b200", "csrc", "ecf8_decode
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
 
 
+HEADLINE = "llama3_70b"
+
+
 def workload_by_name(name: str) -> synth.Workload:
+    if name == HEADLINE:
+        return synth.llama3_70b_layer(0)
     if name == "llama3_8b_layer":
         return synth.llama3_8b_layer()
     if name == "single_1k":
@@ -111,9 +122,11 @@ def kernel_sha() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(workload_name: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source and this workload."""
+def recorded_traffic(workload_name: str, blob_bytes_per_launch=None):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source and this workload.  When the summary records the
+    compressed bytes of its captured launch, the read bytes are scaled to
+    blob_bytes_per_launch (the timed launches' average)."""
     try:
         rec = {}
         with open(TRAFFIC_FILE) as f:
@@ -121,8 +134,12 @@ def recorded_traffic(workload_name: str):
                 if ":" in line and not line.startswith("#"):
                     k, v = line.split(":", 1)
                     rec[k.strip()] = v.strip()
-        if rec.get("kernel_sha") == kernel_sha() and rec.get("workload") == workload_name:
-            return float(rec["dram_bytes_per_launch"])
+        if rec.get("kernel_sha") != kernel_sha() or rec.get("workload") != workload_name:
+            return None
+        if blob_bytes_per_launch is not None and "dram_read_bytes" in rec and "blob_bytes" in rec:
+            read = float(rec["dram_read_bytes"]) * blob_bytes_per_launch / float(rec["blob_bytes"])
+            return round(read + float(rec["dram_write_bytes"]))
+        return float(rec["dram_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -243,11 +260,14 @@ def run_reference(args, workload):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": workload.name, "tensors": len(workload.tensors),
-                   "sample_weights_per_tensor": sample, "ratio_of_sample": summ["ratio"]},
+        "config": {"workload": (f"llama3_70b_{args.layers}layers_reused_buffer" if args.workload == HEADLINE
+                                else workload.name),
+                   "tensors": len(workload.tensors), "sample_weights_per_tensor": sample,
+                   "ratio_of_sample": summ["ratio"]},
         "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"first {sample} weights of each of the {len(xs)} tensors, "
-                                   "one tensor per thread, per step"},
+                         "sample": f"first {sample} weights of each of the {len(xs)} tensors"
+                                   + (" of layer 0" if args.workload == HEADLINE else "")
+                                   + ", one tensor per thread, per step"},
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -701,6 +721,333 @@ def run_bf16(args):
             f.write(json.dumps(line) + "\n")
 
 
+# ---------------------------------------------------------------- headline: the 70B set, 80 layers
+
+_GPU_CHUNK = 1 << 25
+
+
+def _sas_on_gpu(torch, dev, spec):
+    """A tensor of the spec's law drawn on the GPU: symmetric alpha-stable by
+    Chambers, Mallows and Stuck in float64 from torch's Philox generator
+    (seeded from the spec's seed, chunk by chunk), scaled so that max|w| =
+    spec.max_abs, cast to E4M3 (saturating clamp, nearest even).  The same law
+    as the host generator, not the same numbers."""
+    import math
+
+    def chunk_values(c, m):
+        g = torch.Generator(device=dev)
+        g.manual_seed((spec.seed * 1_000_003 + c) & 0x7FFFFFFFFFFFFFFF)
+        u1 = torch.rand(m, dtype=torch.float64, device=dev, generator=g)
+        u2 = torch.rand(m, dtype=torch.float64, device=dev, generator=g)
+        v = math.pi * (u1 - 0.5)
+        w = (-torch.log1p(-u2)).clamp_min(1e-300)
+        a = spec.alpha
+        return torch.sin(a * v) / torch.cos(v).pow(1.0 / a) * (torch.cos(v - a * v) / w).pow((1.0 - a) / a)
+
+    n = spec.n
+    chunks = [(c, min(_GPU_CHUNK, n - c * _GPU_CHUNK)) for c in range((n + _GPU_CHUNK - 1) // _GPU_CHUNK)]
+    mx = max(float(chunk_values(c, m).abs().max()) for c, m in chunks)
+    scale = spec.max_abs / mx
+    out = torch.empty(n, dtype=torch.uint8, device=dev)
+    for c, m in chunks:
+        x = (chunk_values(c, m) * scale).clamp(-448.0, 448.0).to(torch.float32)
+        out[c * _GPU_CHUNK:c * _GPU_CHUNK + m].copy_(x.to(torch.float8_e4m3fn).view(torch.uint8))
+    return out
+
+
+def _encode_set(L, torch, d_xs):
+    """Histogram, codebook and GPU encoding of device tensors: [(info, d_blob)], hists, codebooks."""
+    row, hists, cbs = [], [], []
+    for d in d_xs:
+        h = L.histogram_device(d)
+        cb = L.build_codebook(h)
+        blob = L.encode_device(d, codebook=cb, hist=h)
+        row.append((L.blob_info_device(blob), blob))
+        hists.append(h)
+        cbs.append(cb)
+    return row, hists, cbs
+
+
+def _gen_on_device(torch, dev, specs, world, rank):
+    """Generate the specs' tensors with the host generator (rank 0) and place
+    them on every rank's GPU (a broadcast when there are several ranks);
+    returns the device tensors and, on rank 0, the host arrays."""
+    import torch.distributed as dist
+    xs, d_xs = [], []
+    for t in specs:
+        if rank == 0:
+            x = t.generate()
+            xs.append(x)
+            d = torch.from_numpy(x).to(dev)
+        else:
+            d = torch.empty(t.n, dtype=torch.uint8, device=dev)
+        if world > 1:
+            dist.broadcast(d, 0)
+        d_xs.append(d)
+    return d_xs, xs
+
+
+def _sources(torch, dev, spec_sets, world, rank, host_first=True):
+    """Device tensors for a list of tensor sets: the first set from the host
+    generator (it is what the parity tests decode and what the CPU baseline
+    times), the others drawn on the GPU.  Returns (list of device lists, host
+    arrays of the first set)."""
+    out, xs0 = [], []
+    for k, specs in enumerate(spec_sets):
+        if k == 0 and host_first:
+            d_xs, xs0 = _gen_on_device(torch, dev, specs, world, rank)
+        else:
+            d_xs = [_sas_on_gpu(torch, dev, t) for t in specs]
+        out.append(d_xs)
+    return out, xs0
+
+
+def _layout_outputs(torch, dev, infos):
+    offs, o = [], 0
+    for i in infos:
+        offs.append(o)
+        o += (int(i.n) + 255) // 256 * 256
+    return torch.empty(max(o, 256), dtype=torch.uint8, device=dev), offs
+
+
+def _batch_for(L, row, d_out, out_offs):
+    return L.make_batch([L.BatchItem(info, blob, int(d_out.data_ptr()) + oo)
+                         for (info, blob), oo in zip(row, out_offs)])
+
+
+def _summary(row, hists, cbs):
+    n = sum(int(i.n) for i, _ in row)
+    blob = sum(int(b.numel()) for _, b in row)
+    hist = sum(h.astype(np.float64) for h in hists)
+    bits = sum(int(i.code_bits) for i, _ in row)
+    le6 = sum(float(h[cb.lengths.astype(np.int64) <= 6].sum()) for h, cb in zip(hists, cbs))
+    return {"n_bytes": n, "compressed_bytes": blob, "ratio": round(n / blob, 4),
+            "savings_pct": round(100 * (1 - blob / n), 2), "exponent_entropy_bits": round(entropy_bits(hist), 4),
+            "mean_code_bits": round(bits / n, 4), "codes_le6_bits_frac": round(le6 / n, 5),
+            "max_code_bits": max(int(i.max_len) for i, _ in row)}
+
+
+def _extra_config(L, torch, dev, spec_sets, steps, status, name, peak, note):
+    """One batched launch over every tensor of the spec sets per step: decode
+    GB/s (FP8 out) and roofline fraction, every output checked first."""
+    sets, _ = _sources(torch, dev, spec_sets, 1, 0)
+    d_xs = [d for ds in sets for d in ds]
+    row, hists, cbs = _encode_set(L, torch, d_xs)
+    d_out, out_offs = _layout_outputs(torch, dev, [i for i, _ in row])
+    ws = torch.empty(max(L.batched_workspace_size(len(row)), 16), dtype=torch.uint8, device=dev)
+    batch = _batch_for(L, row, d_out, out_offs)
+    fn = lambda: L.decode_batched(batch, workspace=ws, status=status)  # noqa: E731
+    fn()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"{name}: decode status {int(status.item())}"
+    for k, d_x in enumerate(d_xs):
+        if not torch.equal(d_out[out_offs[k]:out_offs[k] + d_x.numel()], d_x):
+            raise SystemExit(f"{name}: decoded bytes differ from the source (tensor {k})")
+    ms = _time_launches(torch, fn, steps, 3)
+    summ = _summary(row, hists, cbs)
+    alg = summ["compressed_bytes"] + summ["n_bytes"]
+    res = {"workload": name, "tensors": len(row), "launches_per_step": 1, "ms_per_step": round(ms, 5),
+           "gbps_fp8_out": round(summ["n_bytes"] / ms / 1e6, 2),
+           "roofline_frac": round(alg / ms / 1e6 / peak, 4), "note": note, **summ}
+    del row, d_out, ws, d_xs, sets
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_headline(args):
+    """The 70B set: 80 layers compressed-resident, decoded layer by layer into
+    one reused buffer (ECF8 walkthrough §3.2.2: a pool sized for the largest
+    layer, reused), one step = the 80-layer loop."""
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    L = load_library()
+    layers = args.layers
+    specs = synth.llama3_70b_layer(0).tensors
+    # layer 0 from the host generator (the parity tests' tensors), layers
+    # 1..79 drawn on the GPU from their own seeds; every tensor encoded on the
+    # GPU with its own codebook.  The sources (68 GB) stay on the device until
+    # every layer's decode has been compared with them, then are dropped.
+    layer_specs = [synth.llama3_70b_layer(l).tensors for l in range(layers)]
+    sets, xs = _sources(torch, dev, layer_specs[:1], world, rank)
+    rows, hists, cbs, srcs = [], [], [], []
+    for l in range(layers):
+        d_xs = sets[0] if l == 0 else [_sas_on_gpu(torch, dev, t) for t in layer_specs[l]]
+        row, h, cb = _encode_set(L, torch, d_xs)
+        rows.append(row)
+        hists += h
+        cbs += cb
+        srcs.append(d_xs)
+    infos0 = [i for i, _ in rows[0]]
+    d_out, out_offs = _layout_outputs(torch, dev, infos0)  # one buffer, reused by every layer
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    batches = [_batch_for(L, row, d_out, out_offs) for row in rows]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for b in batches:
+            L.decode_batched(b, status=status, stream=stream)
+
+    # correctness of the timed configuration: every layer bit-exact against its source
+    for l, b in enumerate(batches):
+        L.decode_batched(b, status=status, stream=stream)
+        for k in range(len(specs)):
+            if not torch.equal(d_out[out_offs[k]:out_offs[k] + int(infos0[k].n)], srcs[l][k]):
+                raise SystemExit(f"decode mismatch: layer {l} tensor {specs[k].name}")
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"decode status {int(status.item())}"
+    d_xs0 = srcs[0]
+    del srcs, sets
+    torch.cuda.empty_cache()
+
+    n_layer = sum(int(i.n) for i in infos0)
+    blob_layer = sum(int(b.numel()) for b in (blob for _, blob in rows[0]))
+    blob_total = sum(int(b.numel()) for row in rows for _, b in row)
+    n_total = n_layer * layers
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0
+    w = 0
+    while w < args.warmup or time.perf_counter() < t_end:
+        step()
+        w += 1
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches0 = L.launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = L.launch_count() - launches0
+    clk = clocks.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    per_launch_ms = elapsed_ms / max(1, launches)
+    elapsed_ms, per_launch_ms = max_over_ranks([elapsed_ms, per_launch_ms], dev)
+    if world > 1:
+        dist.barrier()
+    assert int(status.item()) == 0
+
+    # end to end through the same call, one layer per step: pinned host blobs
+    # -> device, decode, device -> pinned host output
+    h_blobs, blob_offs, o = [], [], 0
+    for _, b in rows[0]:
+        blob_offs.append(o)
+        o += (int(b.numel()) + 255) // 256 * 256
+    h_blob = torch.empty(o, dtype=torch.uint8, pin_memory=True)
+    d_stage = torch.empty(o, dtype=torch.uint8, device=dev)
+    for (_, b), bo in zip(rows[0], blob_offs):
+        h_blob[bo:bo + b.numel()].copy_(b.cpu())
+    h_out = torch.empty(d_out.numel(), dtype=torch.uint8, pin_memory=True)
+    e2e_batch = L.make_batch([L.BatchItem(info, d_stage[bo:bo + info.blob_bytes], int(d_out.data_ptr()) + oo)
+                              for info, bo, oo in zip(infos0, blob_offs, out_offs)])
+    e2e_steps = max(1, args.e2e_steps)
+
+    def e2e_step():
+        d_stage.copy_(h_blob, non_blocking=True)
+        L.decode_batched(e2e_batch, status=status, stream=stream)
+        h_out.copy_(d_out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
+    out_np = h_out.numpy()
+    for k, d_x in enumerate(d_xs0):
+        if not np.array_equal(out_np[out_offs[k]:out_offs[k] + d_x.numel()], d_x.cpu().numpy()):
+            raise SystemExit("end-to-end decode mismatch")
+    e2e_blob_bytes = sum(int(i.blob_bytes) for i in infos0)
+
+    value = n_total * args.steps * world / (elapsed_ms / 1e3) / 1e9
+    e2e_value = n_layer * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    # one launch = one layer: its compressed bytes read + FP8 bytes written,
+    # averaged over the 80 layers the timed launches decode
+    alg_launch = blob_total / layers + n_layer
+    achieved = alg_launch / (per_launch_ms / 1e3) / 1e9
+    traffic = recorded_traffic("llama3_70b_layer", blob_total / layers)
+    summ = _summary([r for row in rows for r in row], hists, cbs)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        h_blobs = [b.cpu().numpy() for _, b in rows[0]]
+        cpu = oracle_cpu_baseline(h_blobs, xs)
+        del h_blobs
+    del rows, batches, d_stage, h_blob, h_out, d_xs0
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if world == 1 and not args.no_extras:
+        extras["llama3_8b_layer"] = _extra_config(
+            L, torch, dev, [synth.llama3_8b_layer().tensors], max(20, args.steps), status,
+            "llama3_8b_layer_sas1.8", peak, "one batched launch of the 7 tensors (host generator)")
+        moe = synth.moe_experts(args.moe_experts).tensors
+        extras["moe_256x3"] = _extra_config(
+            L, torch, dev, [moe[:3], moe[3:]], max(5, args.steps), status, f"moe_{args.moe_experts}x3_sas1.7",
+            peak, "expert 0 from the host generator, experts 1.. drawn on the GPU from their own seeds; "
+                  "one batched launch of all tensors (workspace)")
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": f"llama3_70b_{layers}layers_reused_buffer",
+                       "description": "Llama-3-70B FP8 weight set: 80 layers x {q,o 8192x8192; k,v 1024x8192; "
+                                      "gate,up 28672x8192; down 8192x28672}, SaS a=1.8, max|w|=448, one codebook "
+                                      "per tensor, compressed-resident, decoded layer by layer into one reused "
+                                      "buffer on one stream",
+                       "layers": layers, "tensors": 7 * layers, "launches_per_step": layers,
+                       "chunk_bytes": int(infos0[0].chunk_bytes), "group_chunks": int(infos0[0].group_chunks),
+                       "resident_compressed_bytes": blob_total, "fp8_bytes_per_step": n_total,
+                       "layer_inputs": "layer 0 from the host generator (the parity tests' tensors); layers 1.. "
+                                       "drawn on the GPU from their own seeds (the same SaS law, torch Philox); "
+                                       "all encoded on the GPU, one codebook per tensor",
+                       "l2": "inputs+outputs larger than L2 (no flush)", **summ},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs", "nominal_peak": NOMINAL_HBM_GBS,
+                         "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "algorithmic_bytes_per_launch": round(alg_launch), "launch_ms": round(per_launch_ms, 5),
+                         "launch": "one layer (7 tensors, one batched decode)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": e2e_blob_bytes,
+                    "d2h_bytes_per_step": int(d_out.numel()), "steps": e2e_steps,
+                    "step": "one layer: pinned host blobs -> device, decode, device -> pinned host"},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "extra": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def load_library(build_only=False):
     from lossless_fp8_weight_b200 import _build
     _build.build()
@@ -714,7 +1061,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama3_8b_layer")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--no-extras", action="store_true", help="headline: leave out the 8B-layer and MoE fields")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--ref-sample", type=int, default=1 << 21)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -742,6 +1090,8 @@ def main():
         return run_encode(args)
     if args.bf16:
         return run_bf16(args)
+    if args.workload == HEADLINE:
+        return run_headline(args)
 
     import torch
     import torch.distributed as dist

@@ -154,12 +154,13 @@ size_t ecf8_encoded_size_bound(size_t n, uint32_t chunk_bytes, uint32_t group_ch
 int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t chunk_bytes,
                 uint32_t group_chunks, void* blob, size_t cap, size_t* blob_bytes);
 
-/* Parse and check a host copy of a blob (the metadata a decoder of the ECF8
+/* Parse and check a blob's header (the metadata a decoder of the ECF8
  * walkthrough §3.2.1 is given beside the bitstream): magic, version, the
  * section layout against n, code_bits, C and T, and the code lengths (a
- * prefix code of at most 16 bits, Kraft sum <= 1).  Reads only the 128-byte
- * header; size is the bytes available at blob.  ECF8_ERR_FORMAT,
- * ECF8_ERR_CODEBOOK. */
+ * prefix code of at most 16 bits, Kraft sum <= 1).  blob (host) must hold at
+ * least the 128-byte header, which is all the call reads; size is the number
+ * of bytes the whole blob occupies where it is stored (host or device), and
+ * must cover the layout's total.  ECF8_ERR_FORMAT, ECF8_ERR_CODEBOOK. */
 int ecf8_blob_info(const void* blob, size_t size, ecf8_info* out);
 
 /* 1 if the GPU kernels implement (chunk_bytes, group_chunks), else 0. */

@@ -267,6 +267,18 @@ def blob_info(blob) -> Info:
     return info
 
 
+def blob_info_device(d_blob) -> Info:
+    """blob_info of a blob held in device memory (a CUDA uint8 tensor): only
+    its 128-byte header is copied to the host, which is all the parser reads."""
+    hdr = np.ascontiguousarray(d_blob[:128].cpu().numpy())
+    if hdr.size < 128:
+        raise Ecf8Error(-2, "ecf8_blob_info")
+    info = Info()
+    _check(_lib.ecf8_blob_info(hdr.ctypes.data, int(d_blob.numel() * d_blob.element_size()), ctypes.byref(info)),
+           "ecf8_blob_info")
+    return info
+
+
 def layout_supported(chunk_bytes: int, group_chunks: int) -> bool:
     return bool(_lib.ecf8_layout_supported(chunk_bytes, group_chunks))
 
