@@ -854,6 +854,40 @@ def _extra_config(L, torch, dev, spec_sets, steps, status, name, peak, note):
     return res
 
 
+def _extra_bf16(L, torch, dev, steps, status, peak):
+    """The BF16 variant (DFloat11 article §3.3 batching): the seven Llama-3-8B
+    projections in BF16 decoded by one batched launch per step, outputs
+    checked first; roofline bytes = blobs read + BF16 written + tables read."""
+    specs = synth.llama3_8b_layer_bf16().tensors
+    xs = [t.generate_bf16() for t in specs]
+    blobs = [L.bf16_encode(x) for x in xs]
+    infos = [L.bf16_blob_info(b) for b in blobs]
+    d_blobs = [torch.from_numpy(b).to(dev) for b in blobs]
+    d_tables = [torch.from_numpy(L.bf16_table(i)).to(dev) for i in infos]
+    d_outs = [torch.empty(int(i.n), dtype=torch.int16, device=dev) for i in infos]
+    items = [(infos[k], d_blobs[k], d_tables[k], d_outs[k]) for k in range(len(specs))]
+    fn = lambda: L.bf16_decode_batched(items, status)  # noqa: E731
+    fn()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"BF16 decode status {int(status.item())}"
+    for x, d in zip(xs, d_outs):
+        if not np.array_equal(d.cpu().numpy().view(np.uint16), x):
+            raise SystemExit("BF16 decode mismatch")
+    launches0 = L.launch_count()
+    ms = _time_launches(torch, fn, steps, 3)
+    launches = (L.launch_count() - launches0) // (steps + 3)
+    n = sum(int(i.n) for i in infos)
+    blob = sum(int(b.size) for b in blobs)
+    alg = blob + 2 * n + len(specs) * int(L._lib.ecf8_bf16_table_bytes())
+    res = {"workload": "bf16_llama3_8b_layer_normal0.02", "tensors": len(specs), "launches_per_step": launches,
+           "ms_per_step": round(ms, 5), "gbps_bf16_out": round(2 * n / ms / 1e6, 2),
+           "roofline_frac": round(alg / ms / 1e6 / peak, 4), "ratio_vs_bf16": round(2 * n / blob, 4),
+           "bits_per_weight": round(8 * blob / n, 4), "n_weights": n, "compressed_bytes": blob}
+    del d_blobs, d_tables, d_outs
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_headline(args):
     """The 70B set: 80 layers compressed-resident, decoded layer by layer into
     one reused buffer (ECF8 walkthrough §3.2.2: a pool sized for the largest
@@ -1010,6 +1044,7 @@ def run_headline(args):
             L, torch, dev, [moe[:3], moe[3:]], max(5, args.steps), status, f"moe_{args.moe_experts}x3_sas1.7",
             peak, "expert 0 from the host generator, experts 1.. drawn on the GPU from their own seeds; "
                   "one batched launch of all tensors (workspace)")
+        extras["bf16_llama3_8b_layer"] = _extra_bf16(L, torch, dev, max(20, args.steps), status, peak)
 
     if rank == 0:
         line = {

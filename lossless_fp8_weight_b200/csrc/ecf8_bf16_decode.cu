@@ -16,7 +16,10 @@
 // it; the next group's stream words are loaded before the current group is
 // processed.  One launch covers up to ECF8_BF16_BATCH_MAX tensors of one
 // layout: each persistent CTA takes a contiguous run of their groups and
-// restages its table where the run crosses into the next tensor.
+// restages its table where the run crosses into the next tensor.  Launches
+// allow programmatic dependent launch: a decode's CTAs may become resident
+// while the previous kernel on the stream drains, and wait for it before they
+// touch global memory.
 //
 // Four table layouts; the host picks wide, byte or narrow per tensor (the
 // lane-private one only when asked for):
@@ -453,9 +456,14 @@ template <int V>
 __global__ void __launch_bounds__(Cfg<V>::kMaxWarps * 32, 1)
     decode_kernel(const __grid_constant__ Batch b, int32_t* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
+  // programmatic dependent launch: the next kernel on the stream may start
+  // its CTAs early; this one touches no global memory (blobs, tables or
+  // outputs the previous kernel may still use) before that kernel completes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t warps = blockDim.x >> 5, warp = threadIdx.x >> 5;
   const uint32_t g_begin = (uint32_t)((uint64_t)b.total_groups * blockIdx.x / gridDim.x);
   const uint32_t g_end = (uint32_t)((uint64_t)b.total_groups * (blockIdx.x + 1) / gridDim.x);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint16_t* zero_codes = reinterpret_cast<const uint16_t*>(smem_raw + b.zc_off);
   WarpArea<V>* wa = reinterpret_cast<WarpArea<V>*>(smem_raw + b.warp_off) + warp;
   uint32_t k = 0;
@@ -518,8 +526,18 @@ int launch(const Args* ts, uint32_t count, int32_t* d_status, cudaStream_t s) {
     return ECF8_ERR_CUDA;
   const uint64_t ctas_needed = (total + warps - 1) / warps;
   const uint32_t grid = (uint32_t)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
-  decode_kernel<V><<<grid, warps * 32, smem, s>>>(b, d_status);
-  if (cudaGetLastError() != cudaSuccess) return ECF8_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(warps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_kernel<V>, b, d_status) != cudaSuccess || cudaGetLastError() != cudaSuccess)
+    return ECF8_ERR_CUDA;
   ecf8::note_launch();
   return ECF8_OK;
 }
