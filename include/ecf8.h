@@ -44,8 +44,11 @@
  *                   offset of the first code start at or after the chunk start
  *                   (the stream end counts as a start), 0 past the end.
  *     group offsets G+1 u64: number of codes starting before bit 8*C*T*g.
- *     code stream   G*T*C bytes + 16 zero bytes; u32 words, stream bit i is
- *                   bit 31-(i%32) of word i/32.
+ *     code stream   G*T*C bytes + 16 zero bytes of u32 words.  Stream bit i
+ *                   is bit 31-(i%32) of reading-order word i/32; inside each
+ *                   group of T chunks, reading-order word m of chunk c is
+ *                   stored at word m*T + c of the group (word-major), so the
+ *                   T decoder threads' word m are adjacent.
  *     nibbles       ceil(n/32)*16 bytes, 8 weights per u32 word w: byte k
  *                   (k = 0..3) holds weight 8w+k's sign in bit 7 and mantissa
  *                   in bits 0-2, weight 8w+4+k's mantissa in bits 4-6, and in

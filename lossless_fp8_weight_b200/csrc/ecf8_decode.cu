@@ -345,17 +345,15 @@ struct GroupIn {
 __device__ __forceinline__ void fetch_group(const DevTensor* dt, uint32_t local, GroupIn& in) {
   const uint32_t lane = threadIdx.x & 31;
   const uint64_t chunk = (uint64_t)local * kT + lane;
-  const uint32_t* stream = dt->stream;
-  const uint4* cs = reinterpret_cast<const uint4*>(stream + chunk * kWords);
+  // inside a group the stream is stored word-major (word m of chunk c at
+  // m * kT + c): the warp's load of word m is 128 contiguous bytes.  A lane's
+  // next word is word 0 of the next chunk, stored right after its own word 0;
+  // lane 31's is word 0 of the next group's first chunk (or the stream's zero
+  // tail after the last group)
+  const uint32_t* gs = dt->stream + (uint64_t)local * (kT * kWords) + lane;
 #pragma unroll
-  for (int q = 0; q < kWords / 4; ++q) {
-    const uint4 v = __ldg(cs + q);
-    in.w[4 * q + 0] = v.x;
-    in.w[4 * q + 1] = v.y;
-    in.w[4 * q + 2] = v.z;
-    in.w[4 * q + 3] = v.w;
-  }
-  in.w[kWords] = __ldg(stream + (chunk + 1) * kWords);
+  for (int m = 0; m < kWords; ++m) in.w[m] = __ldg(gs + m * kT);
+  in.w[kWords] = __ldg(gs + (lane + 1 < (uint32_t)kT ? 1u : (uint32_t)(kT * kWords - lane)));
   in.gapw = __ldg(dt->gaps + (chunk >> 3));
   // the first gap of the next group (lane 31's right neighbour), if it exists
   in.gapn = (lane == 31 && local + 1 < dt->n_groups) ? __ldg(dt->gaps + ((chunk + 1) >> 3)) : 0u;

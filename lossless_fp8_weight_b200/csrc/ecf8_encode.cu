@@ -9,7 +9,8 @@
 //   histogram_kernel   exponent counts (16 per tensor)
 //   seg_bits_kernel    code bits of every 4096-weight segment
 //   scan_kernel        segment start bits (exclusive scan, one CTA)
-//   pack_kernel        the code stream, gaps and group offsets
+//   pack_kernel        the code stream (word-major inside each group), gaps
+//                      and group offsets
 //   tail_kernel        offsets of groups that start past the stream end
 //   nibble_kernel      8 signs and mantissas per 32-bit word
 #include <cuda_runtime.h>
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const uint32_t* seg_
 
 struct PackArgs {
   uint64_t n, code_bits, chunks, chunk_bits;
-  uint32_t T;
+  uint32_t C, T;
   uint32_t* stream;
   uint32_t* gaps;
   uint64_t* offs;
@@ -186,12 +187,13 @@ __global__ void __launch_bounds__(kSegThreads) pack_kernel(const uint8_t* __rest
     if (nacc >= 32) {
       nacc -= 32;
       const uint32_t v = (uint32_t)(acc >> nacc);
-      if (word == first_word) atomicOr(&p.stream[word], v);
-      else p.stream[word] = v;
+      const uint64_t at = stream_word_pos(word, p.C, p.T);
+      if (word == first_word) atomicOr(&p.stream[at], v);
+      else p.stream[at] = v;
       ++word;
     }
   }
-  if (nacc) atomicOr(&p.stream[word], (uint32_t)(acc << (32 - nacc)));  // shared with the next thread
+  if (nacc) atomicOr(&p.stream[stream_word_pos(word, p.C, p.T)], (uint32_t)(acc << (32 - nacc)));  // shared with the next thread
   // the stream end counts as a code start: chunks starting in (last start, end]
   if (i0 + 16 >= p.n) {
     const uint64_t c0 = ((uint64_t)(prev + 1) + p.chunk_bits - 1) / p.chunk_bits;  // first chunk start > prev
@@ -306,6 +308,7 @@ int ecf8_encode_device(const uint8_t* d_fp8, size_t n, const uint64_t hist[16], 
     p.code_bits = L.code_bits;
     p.chunks = L.groups * group_chunks;
     p.chunk_bits = 8ull * chunk_bytes;
+    p.C = chunk_bytes;
     p.T = group_chunks;
     p.stream = reinterpret_cast<uint32_t*>(blob + L.stream_off);
     p.gaps = reinterpret_cast<uint32_t*>(blob + L.gaps_off);

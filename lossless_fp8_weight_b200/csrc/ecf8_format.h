@@ -49,6 +49,19 @@ inline bool compute_layout(uint64_t n, uint64_t code_bits, uint32_t C, uint32_t 
   return true;
 }
 
+// Where the stream's word w (in reading order) is stored: inside each group
+// of T chunks of C bytes the words are kept word-major, word m of chunk c at
+// position m * T + c of the group, so that a warp reading word m of its T
+// chunks reads adjacent words.
+#if defined(__CUDACC__)
+__host__ __device__
+#endif
+inline uint64_t stream_word_pos(uint64_t w, uint32_t C, uint32_t T) {
+  const uint64_t per_chunk = C / 4, per_group = per_chunk * T;
+  const uint64_t g = w / per_group, r = w % per_group;
+  return g * per_group + (r % per_chunk) * T + r / per_chunk;
+}
+
 // Host side of the device encoder (ecf8_host.cpp): checks the codebook
 // against the tensor's histogram and lays the blob out; writes the 128-byte
 // header, the same as ecf8_encode does.

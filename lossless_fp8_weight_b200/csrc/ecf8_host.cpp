@@ -196,9 +196,9 @@ void pack_range(const uint8_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t 
   uint64_t pos = bit0;
   auto flush_word = [&](uint32_t v) {
     if (word == first_word)
-      __atomic_fetch_or(&stream[word], v, __ATOMIC_RELAXED);
+      __atomic_fetch_or(&stream[stream_word_pos(word, C, T)], v, __ATOMIC_RELAXED);
     else
-      stream[word] = v;
+      stream[stream_word_pos(word, C, T)] = v;
     ++word;
   };
   for (size_t i = i0; i < i1; ++i) {
@@ -219,7 +219,7 @@ void pack_range(const uint8_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t 
   }
   if (nacc) {
     const uint32_t v = (uint32_t)(acc << (32 - nacc));
-    __atomic_fetch_or(&stream[word], v, __ATOMIC_RELAXED);  // shared with the next range
+    __atomic_fetch_or(&stream[stream_word_pos(word, C, T)], v, __ATOMIC_RELAXED);  // shared with the next range
   }
   for (; boundary < bit1 && chunk < chunks; boundary += chunk_bits, ++chunk) put_gap(chunk, bit1 - boundary, i1);
 }

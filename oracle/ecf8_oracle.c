@@ -21,7 +21,10 @@
  *    (Larmore and Hirschberg 1990), leaves before packages on equal weight.
  *  - canonical code (RFC 1951 §3.2.2): codes in (length, symbol) order.
  *  - code stream: little-endian 32-bit words, bit i of the stream is bit
- *    31 - (i mod 32) of word i / 32 (MSB first within a word).
+ *    31 - (i mod 32) of word i / 32 (MSB first within a word).  Inside each
+ *    group of T chunks the words are stored word-major: word m of chunk c at
+ *    position m T + c of the group, so that the T threads of a group read
+ *    their chunks' word m from adjacent words.
  *  - chunk c = stream bits [8Cc, 8C(c+1)); gap_c = first code start at or
  *    after 8Cc minus 8Cc, 4 bits per chunk (p1 §3.2.1 gap[tid]).  The end of
  *    the stream (bit code_bits) counts as a start, so a chunk that begins
@@ -193,12 +196,27 @@ int oracle_canonical_codes(const uint8_t* len, uint32_t* code) {
 }
 
 /* ---------- bit access: MSB first inside little-endian 32-bit words ---------- */
-static int get_bit(const uint8_t* stream, uint64_t i) {
-  uint32_t w = rd32(stream + 4 * (i / 32));
+/* The stream section of a blob with its layout: chunks of C bytes, T chunks
+ * per group. */
+typedef struct { uint8_t* base; uint32_t C, T; } stream_t;
+
+/* Byte offset of the 32-bit word that holds stream bit i.  Bit i lies in
+ * word i / 32 of the stream read in order, which is word m of chunk c of
+ * group g; inside a group the words are stored word-major, word m of chunk c
+ * at position m * T + c, so the T chunks' word m sit side by side. */
+static uint64_t word_offset(const stream_t* s, uint64_t i) {
+  uint64_t w = i / 32, per_chunk = s->C / 4, per_group = per_chunk * s->T;
+  uint64_t g = w / per_group, r = w % per_group;
+  uint64_t c = r / per_chunk, m = r % per_chunk;
+  return 4 * (g * per_group + m * s->T + c);
+}
+
+static int get_bit(const stream_t* s, uint64_t i) {
+  uint32_t w = rd32(s->base + word_offset(s, i));
   return (int)((w >> (31 - (i % 32))) & 1u);
 }
-static void set_bit(uint8_t* stream, uint64_t i) {
-  uint8_t* p = stream + 4 * (i / 32);
+static void set_bit(stream_t* s, uint64_t i) {
+  uint8_t* p = s->base + word_offset(s, i);
   wr32(p, rd32(p) | (1u << (31 - (i % 32))));
 }
 
@@ -215,7 +233,7 @@ static int match_code(const uint8_t* len, const uint32_t* code, int (*bit)(const
   return -1;
 }
 
-static int stream_bit(const void* src, uint64_t i) { return get_bit((const uint8_t*)src, i); }
+static int stream_bit(const void* src, uint64_t i) { return get_bit((const stream_t*)src, i); }
 /* ---------- blob layout ---------- */
 typedef struct {
   uint64_t n, code_bits, groups;
@@ -292,7 +310,7 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
   for (int s = 0; s < NSYM; ++s) blob[96 + s] = len[s];
 
   /* code stream, one bit at a time, and the code start positions it implies */
-  uint8_t* stream = blob + L.stream_off;
+  stream_t stream = {blob + L.stream_off, C, T};
   uint8_t* gaps = blob + L.gaps_off;
   uint8_t* offs = blob + L.groups_off;
   uint64_t chunk_bits = 8ull * C, chunks = L.groups * T;
@@ -313,7 +331,7 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
     if (i == n) break;
     int e = oracle_exponent(x[i]);
     for (int b = len[e] - 1; b >= 0; --b) {
-      if ((code[e] >> b) & 1u) set_bit(stream, pos);
+      if ((code[e] >> b) & 1u) set_bit(&stream, pos);
       pos += 1;
     }
   }
@@ -363,12 +381,12 @@ int oracle_decode(const uint8_t* blob, uint64_t size, uint8_t* out, uint64_t n) 
   if (read_layout(blob, size, &L, len) != 0) return -1;
   if (n != L.n) return -2;
   if (oracle_canonical_codes(len, code) != 0) return -1;
-  const uint8_t* stream = blob + L.stream_off;
+  const stream_t stream = {(uint8_t*)(blob + L.stream_off), L.C, L.T};
   const uint8_t* nib = blob + L.nib_off;
   uint64_t pos = 0;
   for (uint64_t i = 0; i < n; ++i) {
     int used = 0;
-    int e = match_code(len, code, stream_bit, stream, pos, L.code_bits - pos, &used);
+    int e = match_code(len, code, stream_bit, &stream, pos, L.code_bits - pos, &used);
     if (e < 0) return -5;
     pos += (uint64_t)used;
     const uint8_t* word = nib + 4 * (i / 8);
@@ -392,7 +410,7 @@ int oracle_check_index(const uint8_t* blob, uint64_t size) {
   uint32_t code[NSYM];
   if (read_layout(blob, size, &L, len) != 0) return -1;
   if (oracle_canonical_codes(len, code) != 0) return -1;
-  const uint8_t* stream = blob + L.stream_off;
+  const stream_t stream = {(uint8_t*)(blob + L.stream_off), L.C, L.T};
   uint64_t chunk_bits = 8ull * L.C, chunks = L.groups * L.T, c = 0, pos = 0;
   for (uint64_t i = 0; i <= L.n + 1; ++i) {
     /* code starts, then the end of the stream, then a start past every chunk */
@@ -407,7 +425,7 @@ int oracle_check_index(const uint8_t* blob, uint64_t size) {
     }
     if (i >= L.n) continue;
     int used = 0;
-    if (match_code(len, code, stream_bit, stream, pos, L.code_bits - pos, &used) < 0) return 4;
+    if (match_code(len, code, stream_bit, &stream, pos, L.code_bits - pos, &used) < 0) return 4;
     pos += (uint64_t)used;
   }
   if (rd64(blob + L.groups_off + 8 * L.groups) != L.n) return 3;

@@ -176,9 +176,16 @@ def test_single_symbol_gets_one_bit():
 # ---------------------------------------------------------------- closed-form streams
 
 def _stream_words(blob):
+    """The stream's words in reading order: within a group the blob keeps
+    word m of chunk c at position m * T + c; this puts them back in order."""
     hd = oracle.blob_header(blob)
+    C, T = hd["chunk_bytes"], hd["group_chunks"]
+    per_chunk = C // 4
+    stored = blob[hd["stream_off"]: hd["stream_off"] + 4 * per_chunk * T * hd["n_groups"]].view("<u4")
+    g, c, m = np.meshgrid(np.arange(hd["n_groups"]), np.arange(T), np.arange(per_chunk), indexing="ij")
+    in_order = stored[(g * per_chunk * T + m * T + c).reshape(-1)]
     words = (hd["code_bits"] + 31) // 32
-    return blob[hd["stream_off"]: hd["stream_off"] + 4 * words].view("<u4"), hd
+    return in_order[:words], hd
 
 
 def test_uniform_16_symbols_stream_is_the_packed_exponents():
@@ -250,6 +257,27 @@ def test_hand_worked_example():
     assert [int(v) for v in nb] == [int(v, 16) for v in g["nibble_bytes"]]
     assert hd["version"] == 2 and hd["reserved"] == 0 and hd["reserved48"] == 0
     assert np.array_equal(oracle.decode(blob, x.size), x)
+
+
+def test_hand_worked_example_word_order_in_groups():
+    """A second hand-derived blob (tests/golden/worked_example_groups.txt) with
+    two words per chunk and two chunks per group, which pins where each stream
+    word is stored inside a group."""
+    g = _read_golden("worked_example_groups.txt")
+    x = np.array([int(v, 16) for v in g["weights"]], dtype=np.uint8)
+    C, T = int(g["chunk_bytes"][0]), int(g["group_chunks"][0])
+    blob = oracle.encode(x, chunk_bytes=C, group_chunks=T)
+    hd = oracle.blob_header(blob)
+    assert list(hd["lengths"]) == [int(v) for v in g["lengths"]]
+    assert hd["code_bits"] == int(g["code_bits"][0]) and hd["n_groups"] == int(g["n_groups"][0])
+    sw = blob[hd["stream_off"]:hd["stream_off"] + 4 * len(g["stored_words"])].view("<u4")
+    assert [int(w) for w in sw] == [int(v, 16) for v in g["stored_words"]]
+    go = blob[hd["groups_off"]:hd["groups_off"] + 8 * (hd["n_groups"] + 1)].view("<u8")
+    assert [int(w) for w in go] == [int(v) for v in g["group_offsets"]]
+    gw = blob[hd["gaps_off"]:hd["gaps_off"] + 4].view("<u4")
+    assert [int(w) for w in gw] == [int(v, 16) for v in g["gap_words"]]
+    assert np.array_equal(oracle.decode(blob, x.size), x)
+    assert oracle.check_index(blob) == 0
 
 
 # ---------------------------------------------------------------- nibble section
