@@ -20,6 +20,12 @@
  *  - length limit binds only below depth 15 (16 leaves): then package-merge
  *    (Larmore and Hirschberg 1990), leaves before packages on equal weight.
  *  - canonical code (RFC 1951 §3.2.2): codes in (length, symbol) order.
+ *  - code order: the stream holds one code per weight, in weight order,
+ *    except that inside every whole block of 8 weights (weights 8b..8b+7,
+ *    all < n) the codes come in the order 8b+0, 8b+4, 8b+1, 8b+5, 8b+2,
+ *    8b+6, 8b+3, 8b+7; a last block of fewer than 8 weights keeps weight
+ *    order.  Code i of the stream is weight coded_weight(i).  ("Code i",
+ *    as in the gaps and group offsets below, counts codes in stream order.)
  *  - code stream: little-endian 32-bit words, bit i of the stream is bit
  *    31 - (i mod 32) of word i / 32 (MSB first within a word).  Inside each
  *    group of T chunks the words are stored word-major: word m of chunk c at
@@ -48,7 +54,7 @@
 #define NSYM 16
 #define HEADER_BYTES 128
 #define MAGIC 0x38464345u /* bytes 'E' 'C' 'F' '8' */
-#define VERSION 2u
+#define VERSION 3u
 
 /* ---------- little-endian field access ---------- */
 static uint32_t rd32(const uint8_t* p) {
@@ -234,6 +240,16 @@ static int match_code(const uint8_t* len, const uint32_t* code, int (*bit)(const
 }
 
 static int stream_bit(const void* src, uint64_t i) { return get_bit((const stream_t*)src, i); }
+/* The weight whose exponent is code i of the stream (see the code order
+ * above): position r = i mod 8 of a whole block holds weight r / 2 of the
+ * block's first half when r is even, weight 4 + r / 2 of its second half
+ * when r is odd. */
+static uint64_t coded_weight(uint64_t i, uint64_t n) {
+  uint64_t block = i / 8, r = i % 8;
+  if (8 * block + 8 > n) return i; /* the last, partial block */
+  return 8 * block + (r % 2 == 0 ? r / 2 : 4 + r / 2);
+}
+
 /* ---------- blob layout ---------- */
 typedef struct {
   uint64_t n, code_bits, groups;
@@ -329,7 +345,7 @@ int oracle_encode(const uint8_t* x, uint64_t n, const uint8_t* len, uint32_t C, 
       next_chunk += 1;
     }
     if (i == n) break;
-    int e = oracle_exponent(x[i]);
+    int e = oracle_exponent(x[coded_weight(i, n)]);
     for (int b = len[e] - 1; b >= 0; --b) {
       if ((code[e] >> b) & 1u) set_bit(&stream, pos);
       pos += 1;
@@ -389,8 +405,9 @@ int oracle_decode(const uint8_t* blob, uint64_t size, uint8_t* out, uint64_t n) 
     int e = match_code(len, code, stream_bit, &stream, pos, L.code_bits - pos, &used);
     if (e < 0) return -5;
     pos += (uint64_t)used;
-    const uint8_t* word = nib + 4 * (i / 8);
-    int r = (int)(i % 8), sign, mant;
+    const uint64_t w = coded_weight(i, n); /* code i is this weight's exponent */
+    const uint8_t* word = nib + 4 * (w / 8);
+    int r = (int)(w % 8), sign, mant;
     if (r < 4) {
       sign = (word[r] >> 7) & 1;
       mant = word[r] & 7;
@@ -398,7 +415,7 @@ int oracle_decode(const uint8_t* blob, uint64_t size, uint8_t* out, uint64_t n) 
       mant = (word[r - 4] >> 4) & 7;
       sign = (word[(r - 3) % 4] >> 3) & 1;
     }
-    out[i] = oracle_join(e, (sign << 3) | mant);
+    out[w] = oracle_join(e, (sign << 3) | mant);
   }
   return pos == L.code_bits ? 0 : -6;
 }

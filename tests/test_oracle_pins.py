@@ -175,6 +175,16 @@ def test_single_symbol_gets_one_bit():
 
 # ---------------------------------------------------------------- closed-form streams
 
+def _weights_in_code_order(n):
+    """Weight index of each code in stream order: every whole block of 8
+    weights contributes its weights 0 4 1 5 2 6 3 7, a last partial block its
+    weights in order."""
+    order = np.arange(n)
+    whole = n // 8 * 8
+    order[:whole] = np.arange(whole) // 8 * 8 + np.tile([0, 4, 1, 5, 2, 6, 3, 7], whole // 8)
+    return order
+
+
 def _stream_words(blob):
     """The stream's words in reading order: within a group the blob keeps
     word m of chunk c at position m * T + c; this puts them back in order."""
@@ -200,7 +210,7 @@ def test_uniform_16_symbols_stream_is_the_packed_exponents():
     words, hd = _stream_words(blob)
     assert list(hd["lengths"]) == [4] * 16
     want = np.zeros(e.size // 8, dtype=np.uint32)
-    for i, v in enumerate(e):
+    for i, v in enumerate(e[_weights_in_code_order(e.size)]):
         want[i // 8] |= np.uint32(int(v) << (28 - 4 * (i % 8)))
     assert np.array_equal(words, want)
     assert np.array_equal(oracle.decode(blob, x.size), x)
@@ -213,7 +223,7 @@ def test_two_symbols_stream_is_a_bitmap():
     blob = oracle.encode(x)
     words, hd = _stream_words(blob)
     assert hd["lengths"][4] == 1 and hd["lengths"][9] == 1
-    bits = "".join("1" if v == 9 else "0" for v in e)
+    bits = "".join("1" if v == 9 else "0" for v in e[_weights_in_code_order(e.size)])
     bits += "0" * (-len(bits) % 32)
     want = np.array([int(bits[i:i + 32], 2) for i in range(0, len(bits), 32)], dtype=np.uint32)
     assert np.array_equal(words, want)
@@ -255,7 +265,7 @@ def test_hand_worked_example():
     assert [int(w) for w in go] == [int(v) for v in g["group_offsets"]]
     nb = blob[hd["nibbles_off"]:hd["nibbles_off"] + 16]
     assert [int(v) for v in nb] == [int(v, 16) for v in g["nibble_bytes"]]
-    assert hd["version"] == 2 and hd["reserved"] == 0 and hd["reserved48"] == 0
+    assert hd["version"] == 3 and hd["reserved"] == 0 and hd["reserved48"] == 0
     assert np.array_equal(oracle.decode(blob, x.size), x)
 
 
@@ -278,6 +288,27 @@ def test_hand_worked_example_word_order_in_groups():
     assert [int(w) for w in gw] == [int(v, 16) for v in g["gap_words"]]
     assert np.array_equal(oracle.decode(blob, x.size), x)
     assert oracle.check_index(blob) == 0
+
+
+def test_code_order_found_by_probing_single_weights():
+    """Where each weight's code sits in the stream, found by probing: all
+    weights but one share exponent 7, the probe has exponent 9, so the two
+    codes are 1 bit long (7 -> 0, 9 -> 1) and the stream is a bitmap with one
+    set bit at the probe's code.  Whole blocks: weight r of a block is code 2r
+    for r < 4 and code 2(r - 4) + 1 for r >= 4; the last partial block keeps
+    weight order."""
+    for n in (8, 20, 23, 24):
+        for k in range(n):
+            x = np.full(n, 0x38, dtype=np.uint8)
+            x[k] = 0x48
+            blob = oracle.encode(x)
+            words, hd = _stream_words(blob)
+            bits = "".join(format(int(w), "032b") for w in words)[: hd["code_bits"]]
+            assert hd["code_bits"] == n and bits.count("1") == 1
+            r = k % 8
+            want = k if k >= n // 8 * 8 else k - r + (2 * r if r < 4 else 2 * (r - 4) + 1)
+            assert bits.index("1") == want, (n, k)
+            assert np.array_equal(oracle.decode(blob, n), x)
 
 
 # ---------------------------------------------------------------- nibble section
@@ -446,7 +477,7 @@ def test_gaps_and_offsets_from_code_start_positions():
         C, T = int(r.choice([4, 8])), int(r.integers(1, 5))
         blob = oracle.encode(x, chunk_bytes=C, group_chunks=T)
         hd = oracle.blob_header(blob)
-        lens = hd["lengths"][(x >> 3) & 15].astype(np.int64)
+        lens = hd["lengths"][(x[_weights_in_code_order(n)] >> 3) & 15].astype(np.int64)
         starts = np.concatenate([[0], np.cumsum(lens)])  # last entry = code_bits
         assert starts[-1] == hd["code_bits"]
         chunks = hd["n_groups"] * T
