@@ -27,10 +27,10 @@
  *    The kernels never read outside [d_blob, d_blob + blob_size), never write
  *    outside [d_out, d_out + n) and never wait.
  *
- * Blob layout (version 2, all fields little-endian; the on-disk and in-HBM
+ * Blob layout (version 3, all fields little-endian; the on-disk and in-HBM
  * form of one compressed tensor):
  *   header, 128 bytes:
- *     0 u32 magic 0x38464345 ("ECF8")   4 u32 version = 2
+ *     0 u32 magic 0x38464345 ("ECF8")   4 u32 version = 3
  *     8 u64 n (weights)                16 u64 code_bits (stream length in bits)
  *    24 u32 chunk_bytes C              28 u32 group_chunks T
  *    32 u32 n_groups G                 36 u32 reserved = 0
@@ -39,6 +39,10 @@
  *    64 u64 offset of group offsets    72 u64 offset of code stream
  *    80 u64 offset of nibbles          88 u64 blob bytes
  *    96 u8[16] code length per exponent value (0 = absent)   112 u8[16] zero
+ *   code order: one code per weight; inside every whole block of 8 weights
+ *     (8b..8b+7 < n) the codes come in the order 8b+0, 8b+4, 8b+1, 8b+5,
+ *     8b+2, 8b+6, 8b+3, 8b+7, and a last block of fewer than 8 weights keeps
+ *     weight order.  "Code i" below counts codes in this stream order.
  *   sections, each at a multiple of 256 bytes, in this order:
  *     gaps          4 bits per chunk, chunk c in bits 4(c%8) of u32 word c/8;
  *                   offset of the first code start at or after the chunk start
@@ -147,7 +151,7 @@ size_t ecf8_encoded_size_bound(size_t n, uint32_t chunk_bytes, uint32_t group_ch
 
 /* Encode n E4M3 bytes into blob (host, capacity cap): the ECF8 walkthrough
  * §3.1.1 steps (exponent field coded with cb, sign and mantissa kept raw)
- * and the per-thread metadata of §3.2.1, in the version-2 layout above.
+ * and the per-thread metadata of §3.2.1, in the version-3 layout above.
  * chunk_bytes is the stream slice of one decoder thread (multiple of 4),
  * group_chunks the chunks that share one group offset.  ECF8_ERR_CODEBOOK if
  * a present exponent has no code or cb's codes are not the canonical code of

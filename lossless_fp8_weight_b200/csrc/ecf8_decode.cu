@@ -281,16 +281,23 @@ __device__ __forceinline__ uint32_t nidx(uint32_t w, uint32_t e, uint32_t k) {
 
 // ---------------------------------------------------------------- assembly
 
-// 8 weights: E = their exponents, 4 bits each in order; N = their nibble
-// word (byte k: weight k's sign in bit 7 and mantissa in bits 0-2, weight
-// 4+k's mantissa in bits 4-6, weight 4+((k+3)%4)'s sign in bit 3), so
-// weights 0-3 take N and weights 4-7 take N rotated right by 4, each masked
-// to bits 7 and 0-2 of every byte.
+// Bits 3-6 of every byte from a, the others from b: one 3-input logic op.
+__device__ __forceinline__ uint32_t merge_exp(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, 0x78787878, 0xE4;" : "=r"(r) : "r"(a), "r"(b));  // (a & c) | (b & ~c)
+  return r;
+}
+
+// 8 weights of a whole block: E = their exponents in stream order, so byte k
+// of E holds weight k's exponent in its low nibble and weight 4+k's in its
+// high nibble; N = their nibble word (byte k: weight k's sign in bit 7 and
+// mantissa in bits 0-2, weight 4+k's mantissa in bits 4-6, weight
+// 4+((k+3)%4)'s sign in bit 3).  Weights 0-3: E << 3 puts each low nibble
+// at bits 3-6, N has the rest in place; weights 4-7: E >> 1 and N rotated
+// right by 4.
 __device__ __forceinline__ void assemble8(uint32_t E, uint32_t N, uint32_t& lo, uint32_t& hi) {
-  const uint32_t ev = (E << 3) & 0x78787878u;  // e0 e2 e4 e6 at bits 3-6 of bytes 0-3
-  const uint32_t od = (E >> 1) & 0x78787878u;  // e1 e3 e5 e7
-  lo = __byte_perm(ev, od, 0x5140) | (N & 0x87878787u);
-  hi = __byte_perm(ev, od, 0x7362) | (__funnelshift_r(N, N, 4) & 0x87878787u);
+  lo = merge_exp(E << 3, N);
+  hi = merge_exp(E >> 1, __funnelshift_r(N, N, 4));
 }
 
 // 32 weights from their exponents (4 words, 8 per word) and nibbles (16
@@ -566,9 +573,12 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     }
   }
   if (hr || tr) {
+    // weight p's code sits at stream position s: the group writes the weights
+    // whose codes it holds, the neighbouring group the others
     const uint64_t p = base + 16ull * ru + (lane & 15);
-    if (rg && p >= off0 && p < off1) {
-      const uint32_t i = 16 * ru + (lane & 15);
+    const uint64_t s = code_position(p, n);
+    if (rg && s >= off0 && s < off1) {
+      const uint32_t i = (uint32_t)(s - base);
       const uint32_t e = (stage[sidx<kW>(i >> 3)] >> (4 * (i & 7))) & 15u;
       const uint32_t k = lane & 7;
       const uint32_t half = k < 4 ? rw : __funnelshift_r(rw, rw, 4);

@@ -9,8 +9,9 @@
 //   histogram_kernel   exponent counts (16 per tensor)
 //   seg_bits_kernel    code bits of every 4096-weight segment
 //   scan_kernel        segment start bits (exclusive scan, one CTA)
-//   pack_kernel        the code stream (word-major inside each group), gaps
-//                      and group offsets
+//   pack_kernel        the code stream (codes of each whole 8-weight block in
+//                      the order 0 4 1 5 2 6 3 7, words word-major inside
+//                      each group), gaps and group offsets
 //   tail_kernel        offsets of groups that start past the stream end
 //   nibble_kernel      8 signs and mantissas per 32-bit word
 #include <cuda_runtime.h>
@@ -153,9 +154,17 @@ __device__ __forceinline__ void put_chunk(const PackArgs& p, uint64_t c, uint64_
 
 __global__ void __launch_bounds__(kSegThreads) pack_kernel(const uint8_t* __restrict__ x, Code c,
                                                            const uint64_t* seg_start, PackArgs p) {
-  uint8_t b[16];
+  uint8_t w[16];
   const uint64_t i0 = (uint64_t)blockIdx.x * kSeg + (uint64_t)threadIdx.x * kPerThread;
-  load16(x, p.n, i0, b);
+  load16(x, p.n, i0, w);
+  // this thread's codes i0 .. i0+15 in stream order: code i0+k is weight
+  // coded_weight(i0+k), one of the thread's own 16 weights
+  uint8_t b[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int r = k & 7, perm = (k & 8) | (r >> 1) | ((r & 1) << 2);
+    b[k] = ((i0 + (k | 7)) < p.n) ? w[perm] : w[k];
+  }
   uint32_t bits = 0;
 #pragma unroll
   for (int k = 0; k < 16; ++k) bits += i0 + k < p.n ? c.len[exponent_of(b[k])] : 0u;
@@ -163,7 +172,8 @@ __global__ void __launch_bounds__(kSegThreads) pack_kernel(const uint8_t* __rest
   const uint32_t incl = cta_inclusive_sum(bits, &total);
   uint64_t pos = seg_start[blockIdx.x] + incl - bits;  // this thread's first code start
   if (i0 >= p.n) return;
-  // start of the previous weight's code (-1 before weight 0)
+  // start of the previous code (-1 before code 0); code i0-1 ends a whole
+  // block, whose last code is its own last weight
   int64_t prev = -1;
   if (i0 > 0) prev = (int64_t)pos - (int64_t)c.len[exponent_of(x[i0 - 1])];
   // pack: MSB first within little-endian 32-bit words

@@ -1,4 +1,4 @@
-// Library-internal constants and layout arithmetic for the ECF8 blob (version 2),
+// Library-internal constants and layout arithmetic for the ECF8 blob (version 3),
 // shared by the host encoder (ecf8_host.cpp) and the decode kernels
 // (ecf8_decode.cu).  The layout itself is documented in include/ecf8.h.
 #pragma once
@@ -10,7 +10,7 @@
 namespace ecf8 {
 
 constexpr uint32_t kMagic = 0x38464345u;  // "ECF8"
-constexpr uint32_t kVersion = 2;
+constexpr uint32_t kVersion = 3;
 constexpr uint32_t kHeaderBytes = 128;
 constexpr uint32_t kSectionAlign = 256;
 
@@ -60,6 +60,28 @@ inline uint64_t stream_word_pos(uint64_t w, uint32_t C, uint32_t T) {
   const uint64_t per_chunk = C / 4, per_group = per_chunk * T;
   const uint64_t g = w / per_group, r = w % per_group;
   return g * per_group + (r % per_chunk) * T + r / per_chunk;
+}
+
+// The weight whose exponent is code i of the stream.  Codes follow the
+// weights, except that inside every whole block of 8 weights they come in the
+// order 0 4 1 5 2 6 3 7: a 32-bit word of 8 decoded exponents then holds
+// weights 0-3 in the low nibbles of its bytes and weights 4-7 in the high
+// ones.  A last block of fewer than 8 weights keeps weight order.
+#if defined(__CUDACC__)
+__host__ __device__
+#endif
+inline uint64_t coded_weight(uint64_t i, uint64_t n) {
+  if ((i | 7) >= n) return i;
+  return (i & ~7ull) | ((i & 7) >> 1) | ((i & 1) << 2);
+}
+
+// The stream position of weight k's code: the inverse of coded_weight.
+#if defined(__CUDACC__)
+__host__ __device__
+#endif
+inline uint64_t code_position(uint64_t k, uint64_t n) {
+  if ((k | 7) >= n) return k;
+  return (k & ~7ull) | ((k & 3) << 1) | ((k >> 2) & 1);
 }
 
 // Host side of the device encoder (ecf8_host.cpp): checks the codebook

@@ -50,13 +50,18 @@ inline uint32_t nibble_word(const uint8_t* b) {
   return v;
 }
 
+// Start of thread range p of `parts` over n weights.  Ranges start on whole
+// 8-weight blocks, so the codes of a range (stream positions [i0, i1)) are the
+// codes of its own weights [i0, i1), only reordered inside blocks.
+size_t range_start(size_t n, int p, int parts) { return p >= parts ? n : (n * (size_t)p / parts) & ~(size_t)7; }
+
 // Per-range exponent histograms, one per thread range, so that the encoder can
 // also derive each range's bit length without a second pass.
 void range_histograms(const uint8_t* x, size_t n, int parts, std::vector<uint64_t>& h) {
   h.assign((size_t)parts * 16, 0);
 #pragma omp parallel for num_threads(parts) schedule(static, 1)
   for (int p = 0; p < parts; ++p) {
-    const size_t i0 = n * (size_t)p / parts, i1 = n * (size_t)(p + 1) / parts;
+    const size_t i0 = range_start(n, p, parts), i1 = range_start(n, p + 1, parts);
     uint64_t c[4][16] = {};
     size_t i = i0;
     for (; i + 4 <= i1; i += 4) {
@@ -175,11 +180,12 @@ bool canonical(const uint8_t* len, uint16_t* code) {
   return true;
 }
 
-// Writes codes [i0, i1) starting at stream bit bit0, and the gap and group
-// offset of every chunk that starts in [bit0, bit1), where bit1 is the start of
-// code i1 (the stream end for the last range).  Words shared with the
-// neighbouring ranges are OR-ed atomically; the stream must start zeroed.
-void pack_range(const uint8_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t bit1, const uint8_t* len,
+// Writes codes [i0, i1) (stream order: code i is weight coded_weight(i, n))
+// starting at stream bit bit0, and the gap and group offset of every chunk
+// that starts in [bit0, bit1), where bit1 is the start of code i1 (the stream
+// end for the last range).  Words shared with the neighbouring ranges are
+// OR-ed atomically; the stream must start zeroed.
+void pack_range(const uint8_t* x, size_t n, size_t i0, size_t i1, uint64_t bit0, uint64_t bit1, const uint8_t* len,
                 const uint16_t* code, uint32_t C, uint32_t T, uint64_t chunks, uint32_t* stream, uint32_t* gaps,
                 uint64_t* offs) {
   const uint64_t chunk_bits = 8ull * C;
@@ -202,7 +208,7 @@ void pack_range(const uint8_t* x, size_t i0, size_t i1, uint64_t bit0, uint64_t 
     ++word;
   };
   for (size_t i = i0; i < i1; ++i) {
-    const uint32_t e = exponent_of(x[i]);
+    const uint32_t e = exponent_of(x[coded_weight(i, n)]);
     if (boundary <= pos && chunk < chunks) {  // at most one boundary per code: codes <= 16 bits <= 8C
       put_gap(chunk, pos - boundary, i);
       ++chunk;
@@ -366,8 +372,8 @@ int ecf8_encode(const uint8_t* fp8, size_t n, const ecf8_codebook* cb, uint32_t 
   const uint64_t chunks = L.groups * group_chunks;
 #pragma omp parallel for num_threads(parts) schedule(static, 1)
   for (int p = 0; p < parts; ++p) {
-    const size_t i0 = n * (size_t)p / parts, i1 = n * (size_t)(p + 1) / parts;
-    pack_range(fp8, i0, i1, range_bit[p], range_bit[p + 1], cb->len, code, chunk_bytes, group_chunks, chunks,
+    const size_t i0 = range_start(n, p, parts), i1 = range_start(n, p + 1, parts);
+    pack_range(fp8, n, i0, i1, range_bit[p], range_bit[p + 1], cb->len, code, chunk_bytes, group_chunks, chunks,
                stream, gaps, offs);
   }
   // a chunk that starts exactly at the stream end, and every later one: gap 0,
