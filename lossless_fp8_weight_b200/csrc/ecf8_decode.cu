@@ -518,11 +518,26 @@ __device__ __forceinline__ void process_group(const DevTensor* dt, uint32_t loca
     uint32_t prev = priv[0];
     if (in_bounds(sidx<kW>(d0) < (uint32_t)kStagePhys, status)) atomicOr(&stage[sidx<kW>(d0)], prev << r);
     uint32_t j = 1;
+    if (kW == kNarrow) {
+      // codes of 2 bits or more: at most 135 per lane, so at most 16
+      // interior words; a fully unrolled, predicated loop
+#pragma unroll
+      for (uint32_t k = 1; k <= 16; ++k) {
+        const uint32_t cur = priv[32 * k];
+        if (k + 1 < nwd && in_bounds(sidx<kW>(d0 + k) < (uint32_t)kStagePhys, status))
+          stage[sidx<kW>(d0 + k)] = __funnelshift_l(prev, cur, r);
+        prev = cur;
+      }
+      j = nwd > 1 ? nwd - 1 : 1;
+      prev = priv[32 * (j - 1)];
+    } else {
 #pragma unroll 4
-    for (; j + 1 < nwd; ++j) {  // interior words belong to this lane alone
-      const uint32_t cur = priv[32 * j];
-      if (in_bounds(sidx<kW>(d0 + j) < (uint32_t)kStagePhys, status)) stage[sidx<kW>(d0 + j)] = __funnelshift_l(prev, cur, r);
-      prev = cur;
+      for (; j + 1 < nwd; ++j) {  // interior words belong to this lane alone
+        const uint32_t cur = priv[32 * j];
+        if (in_bounds(sidx<kW>(d0 + j) < (uint32_t)kStagePhys, status))
+          stage[sidx<kW>(d0 + j)] = __funnelshift_l(prev, cur, r);
+        prev = cur;
+      }
     }
     if (nwd > 1) {
       const uint32_t cur = j < used ? priv[32 * j] : 0;
