@@ -63,6 +63,9 @@ def test_encoder_bytes_equal_oracle_on_hard_inputs(L):
         np.repeat(np.arange(16, dtype=np.uint8) << 3, fib),           # depth-15 code
         np.concatenate([np.zeros(5000, np.uint8), np.full(5000, 0x80, np.uint8)]),  # +-0
         synth.alpha_sweep_point(1.5, 28.0).tensors[0].generate(count=3_000_000),   # mostly 1-bit codes
+        # three encoder thread ranges whose even splits (1,000,001 and 2,000,003)
+        # fall inside 8-weight blocks, and a last block of 5 weights
+        synth.single_normal_1k().tensors[0].generate(count=3_000_005),
     ]
     for x in cases:
         assert np.array_equal(L.encode(x), oracle.encode(x))
