@@ -26,9 +26,9 @@
 //    and subtracted.
 //  * exponents are parked 4 bits each in lane-private shared memory, then
 //    funnel-shifted into a 32-weight-aligned stage; 16 bytes of stage plus a
-//    16-byte nibble load become 32 output bytes (byte-permute + 3-input
-//    logic: the blob's nibble words put each weight's sign and mantissa
-//    where its output byte wants them, or one rotate away), and consecutive
+//    16-byte nibble load become 32 output bytes (per 8 weights two shifts,
+//    a rotate and two 3-input bit-selects: the blob's code order and nibble
+//    words put every field where its output byte wants it), and consecutive
 //    lanes store consecutive 32-byte vectors.
 //  * CTAs are persistent, one per SM.  A launch puts the wide-table tensors on
 //    CTAs [0, split) and the rest on the others; within each part every CTA
