@@ -110,6 +110,24 @@ def test_alpha_stable_prefix(env, alpha, max_abs):
     check_parity(env, spec.generate(count=3_000_001))
 
 
+def test_group_starts_inside_8_weight_blocks(env):
+    """Format 3 orders the codes of each whole 8-weight block 0 4 1 5 2 6 3 7,
+    so a group that starts or ends inside a block owns a scattered subset of
+    the block's weights.  This tensor's group starts fall on every position
+    within a block (checked from the blob's offsets), and the decode must
+    still equal the oracle's byte for byte, ending in a partial last block."""
+    for alpha, max_abs in [(1.7, 448.0), (1.5, 28.0)]:
+        x = synth.alpha_sweep_point(alpha, max_abs).tensors[0].generate(begin=777, count=2_000_003)
+        blob = oracle.encode(x)
+        hd = oracle.blob_header(blob)
+        offs = blob[hd["groups_off"]:hd["groups_off"] + 8 * (hd["n_groups"] + 1)].view("<u8")
+        assert set(int(o) % 8 for o in offs[1:-1]) == set(range(8))
+        got, status, intact = gpu_decode(env, blob)
+        assert status == 0 and intact
+        assert np.array_equal(got, oracle.decode(blob, x.size))
+        assert np.array_equal(got, x)
+
+
 def test_library_blob_decodes_too(env):
     L, _ = env
     x = synth.llama3_8b_layer().tensors[1].generate()
